@@ -1,0 +1,142 @@
+"""Seeded synthetic inputs for the Gated DeltaNet verify / decode / prefill mixer.
+
+This module draws random numbers and rounds them to their storage type; it holds
+none of the mixer's arithmetic. Both the CUDA path's tests / benchmark and the
+CPU oracle take their inputs from here.
+
+Workloads (the shapes of the source pages' target: a 64-layer hybrid whose 48
+Gated DeltaNet layers each carry a 32-bit recurrent state, verified in blocks
+of 7 drafted tokens plus 1 anchor, with a 32K context -- "Qwen 3.8 27B mac m5:
+200 tok/s, audited", sections on fusing layer mixers and on DSpark; and
+"Lithos-metal: Qwen3.8-27B on 40-core M5 Max", quick start, 32K context):
+
+  tiny_verify          B=1,   1 layer,  H_k=H_v=2,   d=16,  T=8, fp32 inputs
+  single_seq_verify    B=1,  48 layers, H_k=16/H_v=48, d=128, T=8, bf16 q/k/v/a/b
+  batched_verify       B=64,  1 layer,  H_k=16/H_v=48, d=128, T=8, bf16
+  decode               B=256, 1 layer,  H_k=16/H_v=48, d=128, T=1, bf16
+  prefill              B=1,   1 layer,  H_k=16/H_v=48, d=128, T=32768, chunk 64, bf16
+
+Distributions: q, k, v, a, b ~ N(0, 1); A_log ~ U(ln 1, ln 16); dt_bias = 0;
+initial state ~ N(0, sigma) with sigma 0.1 (tiny), 0.05 (model-scale), zero for
+prefill; accept_len ~ U{1..8} (tiny) or min(Geometric(0.25), 8) with support
+{1, 2, ...} (model-scale verify). Draw order per (workload, layer) stream:
+S0, q, k, v, a, b, A_log, accept_len. bf16 tensors are rounded once, here,
+round-to-nearest-even, by torch's float32 -> bfloat16 conversion.
+"""
+from dataclasses import dataclass, replace
+from typing import Optional
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    T: int
+    H_k: int
+    H_v: int
+    d_k: int
+    d_v: int
+    layers: int = 1
+    in_dtype: str = "bf16"          # storage type of q, k, v, a, b
+    state_std: float = 0.05         # 0 -> zero initial state
+    accept: str = "geometric"       # "uniform", "geometric", "all" (commit T), "none"
+    chunk: int = 0                  # prefill chunk length (0: not a prefill workload)
+    seed: int = 1000
+
+
+WORKLOADS = {
+    "tiny_verify": Workload("tiny_verify", B=1, T=8, H_k=2, H_v=2, d_k=16, d_v=16,
+                            in_dtype="f32", state_std=0.1, accept="uniform", seed=1000),
+    "single_seq_verify": Workload("single_seq_verify", B=1, T=8, H_k=16, H_v=48, d_k=128,
+                                  d_v=128, layers=48, seed=1001),
+    "batched_verify": Workload("batched_verify", B=64, T=8, H_k=16, H_v=48, d_k=128, d_v=128,
+                               seed=1002),
+    "decode": Workload("decode", B=256, T=1, H_k=16, H_v=48, d_k=128, d_v=128, accept="all",
+                       seed=1003),
+    "prefill": Workload("prefill", B=1, T=32768, H_k=16, H_v=48, d_k=128, d_v=128,
+                        state_std=0.0, accept="none", chunk=64, seed=1004),
+}
+
+# Index of each workload in the list of configurations it was specified as.
+CONFIG_ORDER = ["tiny_verify", "single_seq_verify", "batched_verify", "decode", "prefill"]
+
+
+def workload(name_or_index, **overrides) -> Workload:
+    """A named (or indexed) workload, with optional field overrides (B, T, seed, ...)."""
+    name = CONFIG_ORDER[name_or_index] if isinstance(name_or_index, int) else name_or_index
+    w = WORKLOADS[name]
+    return replace(w, **overrides) if overrides else w
+
+
+def _store(x: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    if dtype == "bf16":
+        return t.to(torch.bfloat16)
+    if dtype == "f32":
+        return t
+    raise ValueError(dtype)
+
+
+def make_inputs(w: Workload, layer: int = 0, gates: str = "config",
+                accept_len: Optional[np.ndarray] = None) -> dict:
+    """Draw one layer's inputs for workload ``w`` (CPU torch tensors).
+
+    gates: "config" (a, b ~ N(0, 1)) or "gentle" (a ~ N(-6, 1): decays near 0.99, so the
+    initial state stays visible in the outputs).
+    Returns q, k [B,T,H_k,d_k]; v [B,T,H_v,d_v]; a, b [B,T,H_v] (in_dtype); A_log, dt_bias
+    [H_v] fp32; S0 [B,H_v,d_v,d_k] fp32; accept_len [B] int32 or None.
+    """
+    rng = np.random.default_rng([w.seed, layer])
+    B, T, Hk, Hv, dk, dv = w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v
+    f32 = np.float32
+    if w.state_std > 0:
+        S0 = rng.standard_normal((B, Hv, dv, dk), dtype=f32) * f32(w.state_std)
+    else:
+        S0 = np.zeros((B, Hv, dv, dk), dtype=f32)
+    q = rng.standard_normal((B, T, Hk, dk), dtype=f32)
+    k = rng.standard_normal((B, T, Hk, dk), dtype=f32)
+    v = rng.standard_normal((B, T, Hv, dv), dtype=f32)
+    a = rng.standard_normal((B, T, Hv), dtype=f32)
+    if gates == "gentle":
+        a = a - f32(6.0)
+    elif gates != "config":
+        raise ValueError(gates)
+    b = rng.standard_normal((B, T, Hv), dtype=f32)
+    A_log = rng.uniform(np.log(1.0), np.log(16.0), size=Hv).astype(f32)
+    dt_bias = np.zeros(Hv, dtype=f32)
+    if accept_len is not None:
+        L = np.ascontiguousarray(accept_len, dtype=np.int32)
+    elif w.accept == "uniform":
+        L = rng.integers(1, T + 1, size=B).astype(np.int32)
+    elif w.accept == "geometric":
+        L = np.minimum(rng.geometric(0.25, size=B), T).astype(np.int32)
+    elif w.accept == "all":
+        L = np.full(B, T, dtype=np.int32)
+    elif w.accept == "none":
+        L = None
+    else:
+        raise ValueError(w.accept)
+    return {
+        "q": _store(q, w.in_dtype), "k": _store(k, w.in_dtype), "v": _store(v, w.in_dtype),
+        "a": _store(a, w.in_dtype), "b": _store(b, w.in_dtype),
+        "A_log": torch.from_numpy(A_log), "dt_bias": torch.from_numpy(dt_bias),
+        "S0": torch.from_numpy(S0),
+        "accept_len": None if L is None else torch.from_numpy(L),
+    }
+
+
+def as_f64(inputs: dict) -> dict:
+    """The same inputs as float64 NumPy arrays (exact: every stored value is representable)."""
+    out = {}
+    for key, val in inputs.items():
+        if val is None:
+            out[key] = None
+        elif key == "accept_len":
+            out[key] = val.numpy().astype(np.int32)
+        else:
+            out[key] = val.to(torch.float64).numpy()
+    return out
+

@@ -1,0 +1,55 @@
+"""Plant plausible mistakes in copies of the oracle's C source and check that the pins in
+test_oracle.py catch every one (a dropped term, a wrong sign or index, a transposed operand,
+an off-by-one commit). Mistakes are planted only in the oracle, on the CPU."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "gdn_oracle.c")
+
+MUTANTS = {
+    "beta_term_sign": ("al * (s - be * p[i] * kt[j])", "al * (s + be * p[i] * kt[j])"),
+    "alpha_dropped": ("al * (s - be * p[i] * kt[j])", "(s - be * p[i] * kt[j])"),
+    "alpha_on_write": ("+ be * vt[i] * kt[j];", "+ al * be * vt[i] * kt[j];"),
+    "output_transposed": ("acc += S[(int64_t)i * dk + j] * qt[j];",
+                          "acc += S[(int64_t)j * dk + i] * qt[j];"),
+    "key_for_query_in_read": ("acc += S[(int64_t)i * dk + j] * qt[j];",
+                              "acc += S[(int64_t)i * dk + j] * kt[j];"),
+    "query_for_key_in_delta": ("acc += S[(int64_t)i * dk + j] * kt[j];",
+                               "acc += S[(int64_t)i * dk + j] * qt[j];"),
+    "gqa_modulo": ("const int g = h / G;\n            int L", "const int g = h % Hk;\n            int L"),
+    "softplus_branch": ("fmax(x, 0.0) + log1p", "fmin(x, 0.0) + log1p"),
+    "sigmoid_sign": ("1.0 / (1.0 + exp(-x))", "1.0 / (1.0 + exp(x))"),
+    "eps_outside_sqrt": ("1.0 / sqrt(ss + eps)", "1.0 / (sqrt(ss) + eps)"),
+    "scale_on_keys": ("oracle_l2norm(nk, dk, k, l2_eps, 1.0, kh)", "oracle_l2norm(nk, dk, k, l2_eps, scale, kh)"),
+    "commit_off_by_one": ("if (t + 1 == L) memcpy", "if (t == L) memcpy"),
+    "A_log_not_exponentiated": ("-exp(A_log[h]) * sp(", "-A_log[h] * sp("),
+    "dt_bias_sign": ("sp(a[idx] + dt_bias[h])", "sp(a[idx] - dt_bias[h])"),
+    "chunk_state_term_sign": ("U[t * dv + i] = Ut[t * dv + i] - ws;", "U[t * dv + i] = Ut[t * dv + i] + ws;"),
+    "chunk_decay_reversed": ("beta[GI(t)] * exp(Gc[t] - Gc[s]) * kk", "beta[GI(t)] * exp(Gc[s] - Gc[t]) * kk"),
+    "chunk_output_diag_dropped": ("for (int s = 0; s <= t; ++s) {\n                        double d = 0.0;",
+                                  "for (int s = 0; s < t; ++s) {\n                        double d = 0.0;"),
+    "chunk_handoff_decay_dropped": ("double acc = eglast * S[(int64_t)i * dk + j];",
+                                    "double acc = S[(int64_t)i * dk + j];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found: " + name
+    mutated = src.replace(old, new, 1)
+    c = tmp_path / "mut.c"
+    c.write_text(mutated)
+    lib = tmp_path / "libmut.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(lib),
+                    str(c), "-lm"], check=True)
+    env = dict(os.environ, GDN_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, r.stdout[-2000:])

@@ -1,0 +1,492 @@
+"""Benchmark of the Gated DeltaNet verify mixer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batched_verify|decode|single_seq_verify|prefill]
+
+A step is one pass of the mixer over one batch of synthetic input, through the C ABI:
+  batched_verify     (default) 64 sequences x 48 value heads, a 7 + 1 verify block, the
+                     committed state written at each sequence's device-side accept count
+  decode             256 sequences, one token each, state updated in place
+  single_seq_verify  one sequence through 48 distinct layers, replayed as a CUDA graph
+  prefill            one 32768-token prompt, chunk 64
+Under torchrun each rank runs its own batch (weak scaling, no data-path collective); the
+step time is the max over ranks. `--impl reference` times the fp64 CPU oracle instead, on
+a bounded sample of the same workload, on rank 0 only.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload  # noqa: E402
+
+METRIC = "GDN verify/decode HBM GB/s (frac of B200 peak), token·heads/s; prefill tok/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["gated_deltanet_mixer_verify_b200/csrc/gdn_verify.cu",
+                  "gated_deltanet_mixer_verify_b200/csrc/gdn_internal.cuh"]
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_name: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or None
+    when there is none for this workload or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(workload_name)
+    if not d or d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def algorithmic_bytes(w, n_state_writes=None):
+    """Bytes one verify / decode call must move: state read + committed state written, the
+    per-token inputs, the gate parameters, the fp32 outputs and the accept counts."""
+    el = 2 if w.in_dtype == "bf16" else 4
+    B, T, Hk, Hv, dk, dv = w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v
+    state = B * Hv * dv * dk * 4
+    writes = B if n_state_writes is None else n_state_writes
+    return (state + writes * Hv * dv * dk * 4 + 2 * B * T * Hk * dk * el + B * T * Hv * dv * el
+            + 2 * B * T * Hv * el + 2 * Hv * 4 + B * T * Hv * dv * 4 + B * 4)
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _sample(self):
+        p = self.nvml
+        self.samples.append(p.nvmlDeviceGetClockInfo(self.h, p.NVML_CLOCK_SM))
+        mask = p.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.nvml:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def workload_config(name):
+    """The JSON `config` of a workload (what it is, with its sizes)."""
+    w = workload(name)
+    c = {"workload": w.name, "B": w.B, "T": w.T, "H_k": w.H_k, "H_v": w.H_v, "d_k": w.d_k,
+         "d_v": w.d_v, "layers": w.layers, "in_dtype": w.in_dtype}
+    if name == "batched_verify":
+        c["accept_len"] = "min(Geometric(0.25), 8) per sequence, device int32"
+        c["state"] = "fp32 [B,H_v,d_v,d_k], committed in place"
+    elif name == "decode":
+        c["state"] = "fp32 [B,H_v,d_v,d_k], updated in place"
+    elif name == "single_seq_verify":
+        c["accept_len"] = "one min(Geometric(0.25), 8) per round, device int32"
+        c["launch"] = "48 launches captured in one CUDA graph"
+    else:
+        c["chunk"] = w.chunk
+        c["state_in"] = "zero"
+    if name == "prefill":
+        c["l2"] = "inputs larger than L2"
+    else:
+        n = algorithmic_bytes(w) * w.layers
+        c["l2"] = "inputs larger than L2 (%.0f MB moved per step, L2 126 MB)" % (n / 1e6)
+    return c
+
+
+class Verify:
+    """batched_verify / decode: one C-ABI call per step over the whole batch."""
+
+    def __init__(self, name, rank, dev):
+        from gated_deltanet_mixer_verify_b200 import gdn
+        self.gdn = gdn
+        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        self.decode = name == "decode"
+        x = make_inputs(self.w)
+        self.host = x
+        self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        self.state = self.x["S0"].clone()
+        self.o = torch.empty(self.x["v"].shape, dtype=torch.float32, device=dev)
+        self.launches_per_step = 1
+        self.bytes = algorithmic_bytes(self.w)
+        self.units = self.w.B * self.w.T * self.w.H_v          # token x heads per step
+
+    def step(self, x=None, o=None):
+        x = x or self.x
+        o = self.o if o is None else o
+        if self.decode:
+            self.gdn.decode_step(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"],
+                                 x["dt_bias"], self.state, o)
+        else:
+            self.gdn.verify_step(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"],
+                                 x["dt_bias"], self.state, self.state, x["accept_len"], o)
+
+    def config(self):
+        return workload_config(self.w.name)
+
+    def per_step_inputs(self):
+        return ["q", "k", "v", "a", "b"] + ([] if self.decode else ["accept_len"])
+
+
+class SingleSeq:
+    """single_seq_verify: one sequence through 48 distinct layers, one launch per layer,
+    captured once as a CUDA graph; a step replays the graph."""
+
+    def __init__(self, name, rank, dev):
+        from gated_deltanet_mixer_verify_b200 import gdn
+        self.gdn = gdn
+        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        L0 = make_inputs(self.w, layer=0)["accept_len"]
+        self.layers = []
+        for l in range(self.w.layers):
+            x = make_inputs(self.w, layer=l, accept_len=L0.numpy())
+            xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+            xd["state"] = xd["S0"].clone()
+            xd["o"] = torch.empty(xd["v"].shape, dtype=torch.float32, device=dev)
+            self.layers.append(xd)
+        self.launches_per_step = self.w.layers
+        self.bytes = algorithmic_bytes(self.w) * self.w.layers
+        self.units = self.w.B * self.w.T * self.w.H_v * self.w.layers
+        self.graph = None
+        self.stream = torch.cuda.Stream(dev)
+
+    def _eager(self):
+        for x in self.layers:
+            self.gdn.verify_step(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"],
+                                 x["dt_bias"], x["state"], x["state"], x["accept_len"], x["o"])
+
+    def step(self):
+        if self.graph is None:
+            with torch.cuda.stream(self.stream):
+                self._eager()                                     # warm the launch path
+            torch.cuda.current_stream().wait_stream(self.stream)
+            torch.cuda.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                self._eager()
+        self.graph.replay()
+
+    def config(self):
+        return workload_config(self.w.name)
+
+
+class Prefill:
+    def __init__(self, name, rank, dev):
+        from gated_deltanet_mixer_verify_b200 import gdn
+        self.gdn = gdn
+        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        x = make_inputs(self.w)
+        self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        w = self.w
+        self.o = torch.empty(self.x["v"].shape, dtype=torch.float32, device=dev)
+        self.state = torch.empty((w.B, w.H_v, w.d_v, w.d_k), dtype=torch.float32, device=dev)
+        nb = gdn.prefill_workspace_bytes(w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v, w.chunk)
+        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        self.launches_per_step = 1
+        el = 2
+        self.bytes = (2 * w.B * w.T * w.H_k * w.d_k * el + w.B * w.T * w.H_v * w.d_v * el
+                      + 2 * w.B * w.T * w.H_v * el + w.B * w.T * w.H_v * w.d_v * 4
+                      + w.B * w.H_v * w.d_v * w.d_k * 4)
+        self.units = w.B * w.T
+
+    def step(self):
+        x = self.x
+        self.gdn.chunk_prefill(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                               None, self.state, self.o, self.w.chunk, self.ws)
+
+    def config(self):
+        return workload_config(self.w.name)
+
+
+WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
+             "prefill": Prefill}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(name, budget_s, rank=0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload's units.
+    Returns (seconds per unit, units timed, description, threads)."""
+    from gated_deltanet_mixer_verify_b200.inputs import as_f64
+    from oracle import gdn_oracle as orc
+    w = workload(name, seed=workload(name).seed + 7919 * rank)
+    threads = orc.max_threads()
+    if name == "prefill":
+        sub = workload(name, T=2048, H_k=1, H_v=3)
+        f = as_f64(make_inputs(sub))
+        t0 = time.perf_counter()
+        orc.prefill(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"], None)
+        dt = time.perf_counter() - t0
+        # units are tokens of all 48 heads: 3 of 48 heads timed over 2048 tokens
+        per_token = dt / 2048 * (w.H_v / 3)
+        return per_token, 2048, "2048 tokens x 3 of 48 value heads (fp64 recurrence)", threads
+    n_seq = {"batched_verify": 8, "decode": 64, "single_seq_verify": 1}[name]
+    sub = workload(name, B=n_seq)
+    f = as_f64(make_inputs(sub))
+    L = f["accept_len"] if name != "decode" else None
+    reps, t_total = 0, 0.0
+    while t_total < budget_s or reps == 0:
+        t0 = time.perf_counter()
+        orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"], f["S0"], L)
+        t_total += time.perf_counter() - t0
+        reps += 1
+        if reps >= 1000:
+            break
+    per_seq = t_total / (reps * n_seq)
+    desc = "%d sequence(s) x %d value heads x T=%d, %d repetition(s)" % (n_seq, w.H_v, w.T, reps)
+    return per_seq, n_seq * reps, desc, threads
+
+
+def cpu_value(name, per_unit_s):
+    """The workload metric (GB/s or tok/s) the oracle reaches at per_unit_s per unit."""
+    w = workload(name)
+    if name == "prefill":
+        return 1.0 / per_unit_s, "tok/s"
+    per_seq_bytes = algorithmic_bytes(workload(name, B=1))
+    return per_seq_bytes / per_unit_s / 1e9, "GB/s"
+
+
+# ----------------------------------------------------------------------------- main
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle as it stands, on the host cores, rank 0 only.
+    Each step is a bounded sample of the workload (one sequence of the batch for verify,
+    16 for decode, 256 tokens x 3 heads for prefill)."""
+    if rank != 0:
+        return
+    from gated_deltanet_mixer_verify_b200.inputs import as_f64
+    from oracle import gdn_oracle as orc
+    name = args.workload
+    if name == "prefill":
+        sub = workload(name, T=256, H_k=1, H_v=3)
+        f = as_f64(make_inputs(sub))
+        run = lambda: orc.prefill(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
+                                  f["dt_bias"], None)
+        units_per_step = 256 * 3 / workload(name).H_v          # prompt tokens (all heads)
+        desc = "256 tokens x 3 of 48 value heads per step (fp64 recurrence)"
+    else:
+        n_seq = 16 if name == "decode" else 1
+        sub = workload(name, B=n_seq)
+        f = as_f64(make_inputs(sub))
+        L = None if name == "decode" else f["accept_len"]
+        run = lambda: orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
+                                 f["dt_bias"], f["S0"], L)
+        units_per_step = algorithmic_bytes(sub) / 1e9          # GB of the workload per step
+        desc = "%d sequence(s) x 48 value heads x T=%d per step" % (n_seq, sub.T)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = units_per_step * args.steps / dt
+    unit = "tok/s" if name == "prefill" else "GB/s"
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": workload_config(name),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": orc.max_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_verify")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import datetime
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = WORKLOADS[args.workload](args.workload, rank, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize(dev)
+
+    # timed region: K steps, device events on the launching stream, per-launch events too
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            wl.step()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+
+    # end to end through the public API: pinned host inputs -> device -> mixer -> host output
+    e2e = None
+    if isinstance(wl, Verify):
+        names = wl.per_step_inputs()
+        host = {k: wl.host[k].pin_memory() for k in names}
+        dev_in = dict(wl.x)
+        dev_in.update({k: torch.empty_like(wl.x[k]) for k in names})
+        o_host = torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+        d2h = o_host.numel() * o_host.element_size()
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e_start.record(stream)
+        for _ in range(args.steps):
+            for k in names:
+                dev_in[k].copy_(host[k], non_blocking=True)
+            wl.step(dev_in)
+            o_host.copy_(wl.o, non_blocking=True)
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = e_start.elapsed_time(e_end)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": wl.bytes * world / (e_ms / args.steps / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        if args.workload == "prefill":
+            value = wl.units * world / (ms_per_step / 1e3)
+            unit = "tok/s"
+        else:
+            value = wl.bytes * world / (ms_per_step / 1e3) / 1e9
+            unit = "GB/s"
+        kernel_ms = statistics.mean(step_ms) / wl.launches_per_step
+        per_launch_bytes = wl.bytes / wl.launches_per_step
+        achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": dict(wl.config(), parallelism="dp%d" % world),
+            "token_heads_per_s": wl.units * world / (ms_per_step / 1e3)
+            if args.workload != "prefill" else None,
+            "frac_of_spec_8TBps": (wl.bytes * world / (ms_per_step / 1e3) / 1e9 / world) / SPEC_HBM_GBS
+            if args.workload != "prefill" else None,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6650 GB/s",
+                         "traffic": ncu_traffic(args.workload),
+                         "algorithmic_bytes_per_launch": per_launch_bytes},
+            "clocks": clk.summary(),
+            "gpu_launches": args.steps * wl.launches_per_step,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            per_unit, units, desc, threads = oracle_sample(args.workload, 10.0)
+            cv, cu = cpu_value(args.workload, per_unit)
+            line["cpu_baseline"] = {"value": cv, "unit": cu, "cores": threads, "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+
+    if isinstance(wl, SingleSeq):
+        wl.graph = None
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -7,7 +7,7 @@ first use, so the input generator works on machines without the built library;
 any call into the mixer raises if the library is missing.
 """
 
-__all__ = ["verify_step", "commit", "decode_step", "chunk_prefill", "stash_bytes",
+__all__ = ["verify_step", "commit", "decode_step", "chunk_prefill", "stash_bytes", "make_shape", "lib",
            "prefill_workspace_bytes", "GdnError", "library_path"]
 
 

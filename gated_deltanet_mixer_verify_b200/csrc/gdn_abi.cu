@@ -1,0 +1,268 @@
+// gdn_abi.cu -- the extern "C" entry points of libgdn.so (declared in include/gdn.h):
+// host-side argument checks, then one kernel launch on the caller's stream.
+// No allocation, no host synchronisation, no copy of device data to the host.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "gdn.h"
+#include "gdn_internal.cuh"
+#include "gdn_prefill.cuh"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+gdn_status fail(gdn_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+gdn_status ok() {
+    g_last_error[0] = '\0';
+    return GDN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dk(int dk) { return dk == 16 || dk == 32 || dk == 64 || dk == 128; }
+
+// Checks common to every call. max_T: largest block length this call supports.
+gdn_status check_shape(const gdn_shape* s, int max_T, const char* who) {
+    if (!s) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
+    if (s->B < 0 || s->T < 1 || s->H_k < 1 || s->H_v < 1 || s->d_k < 1 || s->d_v < 1)
+        return fail(GDN_ERR_INVALID_ARG, "%s: sizes must be positive (B may be 0)", who);
+    if (s->H_v % s->H_k != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: H_v (%d) is not a multiple of H_k (%d)", who, s->H_v, s->H_k);
+    if (s->in_dtype != GDN_F32 && s->in_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "%s: in_dtype %d unknown", who, s->in_dtype);
+    if (s->out_dtype != GDN_F32 && s->out_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "%s: out_dtype %d unknown", who, s->out_dtype);
+    if (!(s->l2_eps >= 0.f) || !(s->scale == s->scale))
+        return fail(GDN_ERR_INVALID_ARG, "%s: l2_eps must be >= 0 and scale a number", who);
+    if (s->B > 65535 || s->H_v > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: B and H_v must be <= 65535", who);
+    if (!supported_dk(s->d_k))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: d_k %d not built (16, 32, 64, 128)", who, s->d_k);
+    if (s->d_v > 4096) return fail(GDN_ERR_UNSUPPORTED, "%s: d_v %d > 4096", who, s->d_v);
+    if (s->T > max_T) return fail(GDN_ERR_UNSUPPORTED, "%s: T %d > %d", who, s->T, max_T);
+    if (s->status_word && !aligned16(s->status_word) &&
+        (reinterpret_cast<uintptr_t>(s->status_word) & 3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: status_word misaligned", who);
+    return GDN_OK;
+}
+
+#define REQUIRE_PTR(p, who)                                                                   \
+    do {                                                                                      \
+        if (!(p)) return fail(GDN_ERR_INVALID_ARG, "%s: %s is NULL", who, #p);                \
+        if (!aligned16(p)) return fail(GDN_ERR_INVALID_ARG, "%s: %s not 16-byte aligned", who, #p); \
+    } while (0)
+
+size_t state_bytes(const gdn_shape* s) {
+    return (size_t)s->B * s->H_v * s->d_v * s->d_k * sizeof(float);
+}
+
+// Distinct or identical, never partially overlapping.
+bool overlap_ok(const void* x, const void* y, size_t bytes) {
+    if (x == y) return true;
+    const char* a = static_cast<const char*>(x);
+    const char* b = static_cast<const char*>(y);
+    return a + bytes <= b || b + bytes <= a;
+}
+
+gdn::VerifyArgs make_args(const gdn_shape* s, const void* q, const void* k, const void* v,
+                          const void* a, const void* b, const float* A_log, const float* dt_bias) {
+    gdn::VerifyArgs x;
+    memset(&x, 0, sizeof(x));
+    x.B = s->B;
+    x.T = s->T;
+    x.Hk = s->H_k;
+    x.Hv = s->H_v;
+    x.dk = s->d_k;
+    x.dv = s->d_v;
+    x.in_bf16 = s->in_dtype == GDN_BF16;
+    x.out_bf16 = s->out_dtype == GDN_BF16;
+    x.q = q;
+    x.k = k;
+    x.v = v;
+    x.a = a;
+    x.b = b;
+    x.A_log = A_log;
+    x.dt_bias = dt_bias;
+    x.l2_eps = s->l2_eps;
+    x.scale = s->scale;
+    x.status_word = s->status_word;
+    return x;
+}
+
+gdn_status launched(cudaError_t e, const char* who) {
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_verify_step(const gdn_shape* shape, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, const float* A_log, const float* dt_bias,
+                           const float* state_in, float* state_out, const int32_t* accept_len,
+                           void* o, float* stash, void* stream) {
+    const char* who = "gdn_verify_step";
+    gdn_status st = check_shape(shape, 16, who);
+    if (st != GDN_OK) return st;
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    REQUIRE_PTR(state_in, who);
+    REQUIRE_PTR(o, who);
+    if (accept_len) {
+        REQUIRE_PTR(accept_len, who);
+        REQUIRE_PTR(state_out, who);
+        if (!overlap_ok(state_in, state_out, state_bytes(shape)))
+            return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
+    } else if (!stash) {
+        return fail(GDN_ERR_INVALID_ARG, "%s: stash is required when accept_len is NULL", who);
+    }
+    if (stash) REQUIRE_PTR(stash, who);
+    gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
+    x.state_in = state_in;
+    x.state_out = accept_len ? state_out : nullptr;
+    x.accept_len = accept_len;
+    x.o = o;
+    x.stash = stash;
+    x.always_commit = 0;
+    return launched(gdn::launch_verify(x, static_cast<cudaStream_t>(stream)), who);
+}
+
+gdn_status gdn_commit(const gdn_shape* shape, const float* state_in, float* state_out,
+                      const float* stash, const int32_t* accept_len, void* stream) {
+    const char* who = "gdn_commit";
+    gdn_status st = check_shape(shape, 16, who);
+    if (st != GDN_OK) return st;
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(state_in, who);
+    REQUIRE_PTR(state_out, who);
+    REQUIRE_PTR(stash, who);
+    REQUIRE_PTR(accept_len, who);
+    if (!overlap_ok(state_in, state_out, state_bytes(shape)))
+        return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
+    gdn::CommitArgs x;
+    x.B = shape->B;
+    x.T = shape->T;
+    x.Hv = shape->H_v;
+    x.dk = shape->d_k;
+    x.dv = shape->d_v;
+    x.state_in = state_in;
+    x.state_out = state_out;
+    x.stash = stash;
+    x.accept_len = accept_len;
+    x.status_word = shape->status_word;
+    return launched(gdn::launch_commit(x, static_cast<cudaStream_t>(stream)), who);
+}
+
+gdn_status gdn_decode_step(const gdn_shape* shape, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, const float* A_log, const float* dt_bias,
+                           float* state, void* o, void* stream) {
+    const char* who = "gdn_decode_step";
+    gdn_status st = check_shape(shape, 1, who);
+    if (st != GDN_OK) return st;
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    REQUIRE_PTR(state, who);
+    REQUIRE_PTR(o, who);
+    gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
+    x.state_in = state;
+    x.state_out = state;
+    x.accept_len = nullptr;
+    x.o = o;
+    x.stash = nullptr;
+    x.always_commit = 1;
+    return launched(gdn::launch_verify(x, static_cast<cudaStream_t>(stream)), who);
+}
+
+size_t gdn_stash_bytes(const gdn_shape* shape) {
+    if (check_shape(shape, 16, "gdn_stash_bytes") != GDN_OK) return 0;
+    return (size_t)shape->B * shape->H_v *
+           gdn::stash_floats_per_head(shape->T, shape->d_k, shape->d_v) * sizeof(float);
+}
+
+size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk) {
+    if (gdn::check_prefill_shape(shape, chunk) != 0) return 0;
+    return gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k, shape->d_v, chunk);
+}
+
+gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,
+                             const void* v, const void* a, const void* b, const float* A_log,
+                             const float* dt_bias, const float* state_in, float* state_out, void* o,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    const char* who = "gdn_chunk_prefill";
+    if (!shape) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
+    gdn_status st = check_shape(shape, 1 << 30, who);
+    if (st != GDN_OK) return st;
+    int pc = gdn::check_prefill_shape(shape, chunk);
+    if (pc != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: only chunk 64 with d_k = d_v = 128 is built", who);
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    REQUIRE_PTR(state_out, who);
+    REQUIRE_PTR(o, who);
+    if (state_in) {
+        REQUIRE_PTR(state_in, who);
+        if (!overlap_ok(state_in, state_out, state_bytes(shape)))
+            return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
+    }
+    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k,
+                                                     shape->d_v, chunk);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", who, need,
+                        workspace_bytes);
+        if (!aligned16(workspace)) return fail(GDN_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", who);
+    }
+    gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
+    x.state_in = state_in;
+    x.state_out = state_out;
+    x.o = o;
+    return launched(gdn::launch_prefill(x, chunk, workspace, workspace_bytes,
+                                        static_cast<cudaStream_t>(stream)),
+                    who);
+}
+
+const char* gdn_status_string(gdn_status status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: bad shape, NULL or misaligned pointer";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: size or type not built into this library";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a kernel launch failed";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "unknown gdn_status";
+}
+
+const char* gdn_last_error(void) { return g_last_error; }
+
+int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,53 @@
+// gdn_internal.cuh -- argument blocks and launcher declarations shared by the C-ABI layer
+// (gdn_abi.cu) and the kernel translation units. Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Arguments of one verify / decode launch (layouts as in include/gdn.h).
+struct VerifyArgs {
+    int B, T, Hk, Hv, dk, dv;
+    int in_bf16, out_bf16;
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* a;
+    const void* b;
+    const float* A_log;
+    const float* dt_bias;
+    const float* state_in;
+    float* state_out;
+    const int32_t* accept_len;   // NULL: no fused commit (two-phase or decode)
+    void* o;
+    float* stash;                // NULL: no stash
+    float l2_eps, scale;
+    int32_t* status_word;
+    int always_commit;           // decode: commit all T tokens, ignore accept_len
+};
+
+// Arguments of the second phase of a two-phase commit.
+struct CommitArgs {
+    int B, T, Hv, dk, dv;
+    const float* state_in;
+    float* state_out;
+    const float* stash;
+    const int32_t* accept_len;
+    int32_t* status_word;
+};
+
+// Stash of one (sequence, value head), in floats: khat [T][d_k], cumulative log-decay
+// G [T] padded to a multiple of 4, then u [T][d_v] padded to a multiple of 4. Every part
+// starts on a 16-byte boundary.
+__host__ __device__ inline size_t stash_floats_per_head(int T, int dk, int dv) {
+    return (size_t)T * dk + (((size_t)T + 3) & ~size_t(3)) + (((size_t)T * dv + 3) & ~size_t(3));
+}
+
+// Host launchers; return cudaSuccess or the launch error. Shapes are validated by the caller.
+cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,204 @@
+"""Thin ctypes binding over libgdn.so (C ABI in include/gdn.h).
+
+Argument marshalling only: every step of the mixer runs in the library's CUDA kernels.
+Tensors are PyTorch CUDA tensors used as device memory; the stream is the current torch
+stream unless one is given. There is no fallback: if libgdn.so is missing or a call fails,
+an exception is raised.
+
+Passages the entry points follow: the Gated DeltaNet mixer and its recurrent-state
+commit / rollback ("Lithos-metal: Qwen3.8-27B on 40-core M5 Max", table "GDN mixer" and
+the runtime paragraph) over a verify block of 7 drafts + 1 anchor ("Qwen 3.8 27B mac m5:
+200 tok/s, audited", DSpark section).
+"""
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+STATUS_BAD_ACCEPT = 1
+
+
+class GdnError(RuntimeError):
+    """A libgdn call returned a non-zero gdn_status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__("gdn status %d: %s" % (status, message))
+        self.status = status
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H_k", ctypes.c_int32),
+                ("H_v", ctypes.c_int32), ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("l2_eps", ctypes.c_float), ("scale", ctypes.c_float),
+                ("status_word", ctypes.c_void_p)]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError("libgdn.so not built at %s: run `python -m gated_deltanet_mixer_verify_b200"
+                          ".build` (or __graft_entry__.build())" % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    S = ctypes.POINTER(_Shape)
+    lib.gdn_verify_step.argtypes = [S] + [_VP] * 13
+    lib.gdn_commit.argtypes = [S] + [_VP] * 5
+    lib.gdn_decode_step.argtypes = [S] + [_VP] * 10
+    lib.gdn_chunk_prefill.argtypes = ([S, ctypes.c_int32] + [_VP] * 11 + [ctypes.c_size_t, _VP])
+    for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill"):
+        getattr(lib, fn).restype = ctypes.c_int
+    lib.gdn_stash_bytes.argtypes = [S]
+    lib.gdn_stash_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_prefill_workspace_bytes.argtypes = [S, ctypes.c_int32]
+    lib.gdn_chunk_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_last_error.argtypes = []
+    lib.gdn_last_error.restype = ctypes.c_char_p
+    lib.gdn_abi_version.argtypes = []
+    lib.gdn_abi_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def lib():
+    """The loaded ctypes library (raises ImportError if it was never built)."""
+    return _load()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise GdnError(rc, _load().gdn_last_error().decode())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return GDN_F32
+    if dt == torch.bfloat16:
+        return GDN_BF16
+    raise TypeError("unsupported dtype %s (float32 or bfloat16)" % dt)
+
+
+def make_shape(B, T, H_k, H_v, d_k, d_v, in_dtype=torch.bfloat16, out_dtype=torch.float32,
+               l2_eps=1e-6, scale=1.0, status_word: Optional[torch.Tensor] = None) -> _Shape:
+    sw = status_word.data_ptr() if status_word is not None else None
+    return _Shape(B, T, H_k, H_v, d_k, d_v, _dtype_code(in_dtype), _dtype_code(out_dtype),
+                  float(l2_eps), float(scale), sw)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype) -> _Shape:
+    B, T, H_k, d_k = k.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    if q.shape != k.shape or v.shape[:2] != (B, T):
+        raise ValueError("q, k [B,T,H_k,d_k] and v [B,T,H_v,d_v] disagree")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    return make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
+
+
+def stash_bytes(B, T, H_k, H_v, d_k, d_v) -> int:
+    """Bytes of stash a two-phase verify writes for this shape."""
+    return int(_load().gdn_stash_bytes(ctypes.byref(make_shape(B, T, H_k, H_v, d_k, d_v))))
+
+
+def prefill_workspace_bytes(B, T, H_k, H_v, d_k, d_v, chunk=64) -> int:
+    """Bytes of workspace gdn_chunk_prefill needs for this shape."""
+    return int(_load().gdn_chunk_prefill_workspace_bytes(
+        ctypes.byref(make_shape(B, T, H_k, H_v, d_k, d_v)), chunk))
+
+
+def verify_step(q, k, v, a, b, A_log, dt_bias, state_in, state_out=None, accept_len=None, o=None,
+                stash=None, l2_eps=1e-6, scale=1.0, status_word=None, out_dtype=torch.float32,
+                stream=None):
+    """One verify block: o for all T tokens; with ``accept_len`` the committed state S_L goes
+    to ``state_out`` (default: in place into ``state_in``); without it, ``stash`` (a float32
+    CUDA tensor of stash_bytes()/4 elements) receives what :func:`commit` needs. Returns o."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    if accept_len is not None and state_out is None:
+        state_out = state_in
+    _check(_load().gdn_verify_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                   _ptr(A_log), _ptr(dt_bias), _ptr(state_in), _ptr(state_out),
+                                   _ptr(accept_len), _ptr(o), _ptr(stash), _stream(stream)))
+    return o
+
+
+def commit(state_in, stash, accept_len, T, H_k, d_k=None, state_out=None, status_word=None,
+           stream=None):
+    """Second phase of a two-phase verify: state_out = S_L from state_in and the stash.
+    ``T`` and ``H_k`` are the verify call's; state_out defaults to state_in (in place)."""
+    B, H_v, d_v, dk = state_in.shape
+    sh = make_shape(B, T, H_k, H_v, dk if d_k is None else d_k, d_v, status_word=status_word)
+    if state_out is None:
+        state_out = state_in
+    _check(_load().gdn_commit(ctypes.byref(sh), _ptr(state_in), _ptr(state_out), _ptr(stash),
+                              _ptr(accept_len), _stream(stream)))
+    return state_out
+
+
+def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale=1.0,
+                status_word=None, out_dtype=torch.float32, stream=None):
+    """One plain decoding token (T = 1): returns o and updates ``state`` in place."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    _check(_load().gdn_decode_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                   _ptr(A_log), _ptr(dt_bias), _ptr(state), _ptr(o),
+                                   _stream(stream)))
+    return o
+
+
+def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, o=None, chunk=64,
+                  workspace=None, l2_eps=1e-6, scale=1.0, status_word=None,
+                  out_dtype=torch.float32, stream=None):
+    """The mixer over a whole prompt: returns (o, state_out). ``state_in`` None = zero state.
+    ``workspace`` (uint8 CUDA tensor) must hold prefill_workspace_bytes(); it is allocated
+    here when not given."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    B, T, H_k, d_k = k.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    if state_out is None:
+        state_out = torch.empty((B, H_v, d_v, d_k), dtype=torch.float32, device=v.device)
+    need = int(_load().gdn_chunk_prefill_workspace_bytes(ctypes.byref(sh), chunk))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_load().gdn_chunk_prefill(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                     _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state_in),
+                                     _ptr(state_out), _ptr(o), _ptr(workspace), wbytes,
+                                     _stream(stream)))
+    return o, state_out

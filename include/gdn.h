@@ -1,0 +1,176 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet layer mixer for speculative
+ * verification, decode and long-prompt prefill on NVIDIA B200 (sm_100a).
+ *
+ * The operation (source pages: "Lithos-metal: Qwen3.8-27B on 40-core M5 Max",
+ * table "GDN mixer" -- the recurrent state is split by value columns and each
+ * slice is kept on-chip across the input block -- and its runtime paragraph,
+ * where the GPU tracks recurrent-state commit and rollback; "Qwen 3.8 27B mac
+ * m5: 200 tok/s, audited", section "How does lithos-metal fuse layer mixers on
+ * Metal?" (a 32-bit recurrent state with a key side and a value side, which a
+ * conventional kernel reads and writes for every token) and section "How does
+ * DSpark speculative decoding create more than one token per read?" (7 drafted
+ * tokens plus 1 anchor are verified as 8 rows; rewind follows acceptance)):
+ *
+ *   for each sequence b and value head h (key head g = h / (H_v / H_k)):
+ *     khat_t = k_t / sqrt(|k_t|^2 + l2_eps),  qhat_t = scale * q_t / sqrt(|q_t|^2 + l2_eps)
+ *     alpha_t = exp(-exp(A_log[h]) * softplus(a_t + dt_bias[h])),  beta_t = sigmoid(b_t)
+ *     S_t = alpha_t S_{t-1} (I - beta_t khat_t khat_t^T) + beta_t v_t khat_t^T
+ *     o_t = S_t qhat_t
+ *   and the state committed for the block is S_L, L = accept_len[b] (L = 0: S_0).
+ *
+ * Layouts (all row-major, contiguous, no padding):
+ *   q, k      [B][T][H_k][d_k]   in_dtype
+ *   v         [B][T][H_v][d_v]   in_dtype
+ *   a, b      [B][T][H_v]        in_dtype   (gate pre-activations)
+ *   A_log     [H_v] fp32,  dt_bias [H_v] fp32
+ *   state     [B][H_v][d_v][d_k] fp32       (row i = value index, column j = key index)
+ *   o         [B][T][H_v][d_v]   out_dtype
+ *   accept_len[B] int32, on the device
+ *
+ * Conventions shared by every call:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *     allocates nothing, frees nothing and keeps no device memory between calls.
+ *     All tensor pointers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream). No call synchronises the host, and no call
+ *     copies accept_len (or anything else) to the host.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     returned as GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED; nothing is written.
+ *     GDN_ERR_CUDA means a launch failed (cudaGetLastError after the launch).
+ *     gdn_last_error() gives a one-line reason for the last failure on the
+ *     calling host thread.
+ *   - Device-side conditions never trap: an accept_len[b] outside 0..T commits
+ *     nothing for sequence b (its state_out equals state_in) and sets bit 0
+ *     (GDN_STATUS_BAD_ACCEPT) of *status_word when status_word is not NULL.
+ *   - Calls that overlap on the GPU and write the same buffers race; calls on
+ *     one stream are ordered.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1,   /* bad shape, NULL or misaligned pointer, H_v % H_k != 0 */
+    GDN_ERR_UNSUPPORTED = -2,   /* valid but not built: d_k / d_v / T / chunk outside the table */
+    GDN_ERR_CUDA = -3,          /* a kernel launch failed */
+    GDN_ERR_WORKSPACE = -4      /* workspace missing or smaller than the size query returns */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Bits the kernels OR into *status_word. */
+#define GDN_STATUS_BAD_ACCEPT 1
+
+/*
+ * Problem description shared by all calls. Sizes supported by this build:
+ *   B in 1..65535, H_v a multiple of H_k, H_v <= 65535,
+ *   d_k in {16, 32, 64, 128, 256}, d_v in 1..4096,
+ *   verify: T in 1..16; decode: T == 1; prefill: T >= 1, chunk == 64, d_k == d_v == 128.
+ */
+typedef struct {
+    int32_t B, T, H_k, H_v, d_k, d_v;
+    int32_t in_dtype;        /* gdn_dtype of q, k, v, a, b */
+    int32_t out_dtype;       /* gdn_dtype of o */
+    float l2_eps;            /* inside the square root of the q/k normalisation, e.g. 1e-6 */
+    float scale;             /* multiplies qhat, e.g. 1.0 or 1/sqrt(d_k) */
+    int32_t* status_word;    /* device int32 or NULL; bits GDN_STATUS_* are OR-ed in */
+} gdn_shape;
+
+/*
+ * gdn_verify_step -- one mixer pass over a verify block of T tokens (7 drafts +
+ * 1 anchor is T = 8; the anchor is token 0), followed by the state commit.
+ * Passages: the "GDN mixer" table and runtime paragraph of "Lithos-metal:
+ * Qwen3.8-27B on 40-core M5 Max"; the DSpark section of "Qwen 3.8 27B mac m5:
+ * 200 tok/s, audited" (8 verify rows, rewind after every acceptance decision).
+ *
+ *   o           out: o_t for all T tokens (outputs never depend on the commit point).
+ *   accept_len  device [B] or NULL.
+ *     non-NULL: fused commit. state_out[b] = S_L with L = accept_len[b]; L = 0 rolls
+ *               back (state_out[b] = state_in[b] bit for bit; when state_out ==
+ *               state_in nothing is written). state_out must not be NULL.
+ *     NULL:     two-phase commit. The accept count is not known yet: stash receives
+ *               what gdn_commit needs and state_out is not written (may be NULL).
+ *   state_out   may equal state_in (in place); partial overlap is not allowed.
+ *   stash       device, gdn_stash_bytes(shape) bytes; required when accept_len is NULL,
+ *               optional (NULL or written) otherwise.
+ */
+gdn_status gdn_verify_step(const gdn_shape* shape,
+                           const void* q, const void* k, const void* v,
+                           const void* a, const void* b,
+                           const float* A_log, const float* dt_bias,
+                           const float* state_in, float* state_out,
+                           const int32_t* accept_len,
+                           void* o, float* stash, void* stream);
+
+/*
+ * gdn_commit -- second phase of a two-phase verify: once the accept count is known on
+ * the device, state_out[b] = S_L built from the block's initial state and the stash
+ * that gdn_verify_step wrote (accept_len NULL). Same passages as gdn_verify_step
+ * (commit / rollback at the accepted prefix; rewind after acceptance).
+ *   state_in   the state gdn_verify_step started from (unchanged since).
+ *   state_out  may equal state_in. L = 0, or L out of range, leaves state_in's values.
+ *   shape      the same shape that was passed to gdn_verify_step.
+ */
+gdn_status gdn_commit(const gdn_shape* shape, const float* state_in, float* state_out,
+                      const float* stash, const int32_t* accept_len, void* stream);
+
+/*
+ * gdn_decode_step -- plain decoding, one token (shape->T must be 1): o = S_1 q and the
+ * state is updated in place (always committed). This is the case the pages describe as
+ * a conventional kernel reading and writing the whole state for every token ("Qwen 3.8
+ * 27B mac m5: 200 tok/s, audited", section on fusing layer mixers).
+ */
+gdn_status gdn_decode_step(const gdn_shape* shape,
+                           const void* q, const void* k, const void* v,
+                           const void* a, const void* b,
+                           const float* A_log, const float* dt_bias,
+                           float* state, void* o, void* stream);
+
+/*
+ * gdn_chunk_prefill -- the mixer over a long prompt (T tokens per sequence), in the
+ * chunked WY / UT-transform form on tensor cores: o for every token and the state after
+ * the last token. The pages time whole-model prefill only ("Qwen 3.8 27B mac m5: 200
+ * tok/s, audited", section "What does long-context prefill cost on Apple silicon?");
+ * the recurrence is the one above.
+ *   state_in   NULL = zero initial state.
+ *   state_out  required; may equal state_in.
+ *   workspace  device scratch of at least gdn_chunk_prefill_workspace_bytes(shape, chunk)
+ *              bytes (16-byte aligned); contents on entry are ignored.
+ */
+gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
+                             const void* q, const void* k, const void* v,
+                             const void* a, const void* b,
+                             const float* A_log, const float* dt_bias,
+                             const float* state_in, float* state_out, void* o,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of stash gdn_verify_step writes for this shape (0 for an invalid shape). */
+size_t gdn_stash_bytes(const gdn_shape* shape);
+
+/* Bytes of workspace gdn_chunk_prefill needs (0 for an invalid shape or chunk). */
+size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk);
+
+/* Static description of a status code. */
+const char* gdn_status_string(gdn_status status);
+
+/* One-line reason for the most recent failing call on this host thread ("" if none). */
+const char* gdn_last_error(void);
+
+/* GDN_ABI_VERSION of the built library. */
+int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,95 @@
+"""The C-ABI library loads without a GPU, exports every entry point include/gdn.h declares,
+and rejects bad arguments on the host before any launch (these calls compute nothing)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_mixer_verify_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def gdn():
+    gbuild.build()
+    from gated_deltanet_mixer_verify_b200 import gdn as g
+    return g
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(gdn):
+    names = declared_functions()
+    assert {"gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill"} <= set(names)
+    lib = gdn.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings(gdn):
+    lib = gdn.lib()
+    assert lib.gdn_abi_version() == 1
+    for code in (0, -1, -2, -3, -4):
+        assert lib.gdn_status_string(code).decode().startswith("GDN_")
+    assert "unknown" in lib.gdn_status_string(7).decode()
+
+
+def test_stash_bytes_formula(gdn):
+    # khat [T][d_k] + G [T pad 4] + u [T*d_v pad 4] floats per (sequence, value head)
+    def per_head(T, dk, dv):
+        pad = lambda x: (x + 3) // 4 * 4
+        return T * dk + pad(T) + pad(T * dv)
+    assert gdn.stash_bytes(64, 8, 16, 48, 128, 128) == 64 * 48 * per_head(8, 128, 128) * 4
+    assert gdn.stash_bytes(1, 3, 1, 1, 16, 5) == per_head(3, 16, 5) * 4
+    assert gdn.stash_bytes(1, 17, 1, 1, 16, 16) == 0          # T > 16: not a verify shape
+
+
+def _call_verify(gdn, shape, ptrs=None, accept=True):
+    p = ptrs or {}
+    fake = 0x10000
+    get = lambda k: p.get(k, fake)
+    return gdn.lib().gdn_verify_step(
+        ctypes.byref(shape) if shape is not None else None, get("q"), get("k"), get("v"), get("a"),
+        get("b"), get("A_log"), get("dt_bias"), get("state_in"), get("state_out"),
+        get("accept_len") if accept else None, get("o"), p.get("stash"), None)
+
+
+def test_host_validation_rejects_before_launch(gdn):
+    INVALID, UNSUP = -1, -2
+    ok_shape = lambda **kw: gdn.make_shape(**dict(dict(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128), **kw))
+    assert _call_verify(gdn, None) == INVALID
+    assert _call_verify(gdn, ok_shape(H_v=47)) == INVALID             # H_v % H_k
+    assert _call_verify(gdn, ok_shape(T=0)) == INVALID
+    assert _call_verify(gdn, ok_shape(B=-1)) == INVALID
+    assert _call_verify(gdn, ok_shape(d_k=96)) == UNSUP
+    assert _call_verify(gdn, ok_shape(T=17)) == UNSUP
+    assert _call_verify(gdn, ok_shape(), {"q": None}) == INVALID      # NULL tensor
+    assert "q is NULL" in gdn.lib().gdn_last_error().decode()
+    assert _call_verify(gdn, ok_shape(), {"v": 0x10008}) == INVALID   # misaligned
+    assert "not 16-byte aligned" in gdn.lib().gdn_last_error().decode()
+    # two-phase without a stash
+    assert _call_verify(gdn, ok_shape(), accept=False) == INVALID
+    # partial overlap of state_out with state_in
+    assert _call_verify(gdn, ok_shape(), {"state_in": 0x100000, "state_out": 0x100010}) == INVALID
+    # decode needs T == 1
+    lib = gdn.lib()
+    sh = ok_shape(T=2)
+    assert lib.gdn_decode_step(ctypes.byref(sh), *([0x10000] * 9), None) == UNSUP
+    # prefill: only chunk 64 with d = 128 is built; workspace checked
+    sh = ok_shape(T=4096)
+    assert lib.gdn_chunk_prefill(ctypes.byref(sh), 32, *([0x10000] * 11), 0, None) == UNSUP
+    sh = ok_shape(T=4096, d_k=64, d_v=64)
+    assert lib.gdn_chunk_prefill(ctypes.byref(sh), 64, *([0x10000] * 11), 0, None) == UNSUP
+
+
+def test_empty_batch_is_a_no_op(gdn):
+    sh = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    assert gdn.lib().gdn_verify_step(ctypes.byref(sh), *([None] * 12), None) == 0
+    assert gdn.lib().gdn_commit(ctypes.byref(sh), None, None, None, None, None) == 0

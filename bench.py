@@ -28,6 +28,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from gated_deltanet_mixer_verify_b200.dist import max_over_ranks, rank_seed, weak_scaling_throughput  # noqa: E402
 from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload  # noqa: E402
 
 METRIC = "GDN verify/decode HBM GB/s (frac of B200 peak), token·heads/s; prefill tok/s"
@@ -163,7 +164,7 @@ class Verify:
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
         self.gdn = gdn
-        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
         self.decode = name == "decode"
         x = make_inputs(self.w)
         self.host = x
@@ -198,7 +199,7 @@ class SingleSeq:
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
         self.gdn = gdn
-        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
         L0 = make_inputs(self.w, layer=0)["accept_len"]
         self.layers = []
         for l in range(self.w.layers):
@@ -237,7 +238,7 @@ class Prefill:
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
         self.gdn = gdn
-        self.w = workload(name, seed=workload(name).seed + 7919 * rank)
+        self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
         x = make_inputs(self.w)
         self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
         w = self.w
@@ -272,7 +273,7 @@ def oracle_sample(name, budget_s, rank=0):
     Returns (seconds per unit, units timed, description, threads)."""
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    w = workload(name, seed=workload(name).seed + 7919 * rank)
+    w = workload(name, seed=rank_seed(workload(name).seed, rank))
     threads = orc.max_threads()
     if name == "prefill":
         sub = workload(name, T=2048, H_k=1, H_v=3)
@@ -407,12 +408,8 @@ def main():
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end))
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     ms_per_step = elapsed_ms / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> mixer -> host output
@@ -437,21 +434,18 @@ def main():
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = e_start.elapsed_time(e_end)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": wl.bytes * world / (e_ms / args.steps / 1e3) / 1e9, "unit": "GB/s",
+        e_ms = max_over_ranks(e_start.elapsed_time(e_end))
+        e2e = {"value": weak_scaling_throughput(wl.bytes, world, e_ms / args.steps / 1e3) / 1e9,
+               "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
         if args.workload == "prefill":
-            value = wl.units * world / (ms_per_step / 1e3)
+            value = weak_scaling_throughput(wl.units, world, ms_per_step / 1e3)
             unit = "tok/s"
         else:
-            value = wl.bytes * world / (ms_per_step / 1e3) / 1e9
+            value = weak_scaling_throughput(wl.bytes, world, ms_per_step / 1e3) / 1e9
             unit = "GB/s"
         kernel_ms = statistics.mean(step_ms) / wl.launches_per_step
         per_launch_bytes = wl.bytes / wl.launches_per_step

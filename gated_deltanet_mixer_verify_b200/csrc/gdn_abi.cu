@@ -44,8 +44,8 @@ gdn_status check_shape(const gdn_shape* s, int max_T, const char* who) {
         return fail(GDN_ERR_INVALID_ARG, "%s: out_dtype %d unknown", who, s->out_dtype);
     if (!(s->l2_eps >= 0.f) || !(s->scale == s->scale))
         return fail(GDN_ERR_INVALID_ARG, "%s: l2_eps must be >= 0 and scale a number", who);
-    if (s->B > 65535 || s->H_v > 65535)
-        return fail(GDN_ERR_UNSUPPORTED, "%s: B and H_v must be <= 65535", who);
+    if (s->B > 65535 || s->H_v > 65535 || (int64_t)s->B * s->H_v > (1 << 24))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: B, H_v <= 65535 and B * H_v <= 2^24 required", who);
     if (!supported_dk(s->d_k))
         return fail(GDN_ERR_UNSUPPORTED, "%s: d_k %d not built (16, 32, 64, 128)", who, s->d_k);
     if (s->d_v > 4096) return fail(GDN_ERR_UNSUPPORTED, "%s: d_v %d > 4096", who, s->d_v);
@@ -245,6 +245,7 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* 
     x.state_in = state_in;
     x.state_out = state_out;
     x.o = o;
+    x.always_commit = 1;   // the state after the last prompt token is always written
     return launched(gdn::launch_prefill(x, chunk, workspace, workspace_bytes,
                                         static_cast<cudaStream_t>(stream)),
                     who);

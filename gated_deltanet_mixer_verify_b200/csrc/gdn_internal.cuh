@@ -27,6 +27,7 @@ struct VerifyArgs {
     float l2_eps, scale;
     int32_t* status_word;
     int always_commit;           // decode: commit all T tokens, ignore accept_len
+    int row_split;               // head kernel: CTAs (work items) per head, set by its launcher
 };
 
 // Arguments of the second phase of a two-phase commit.
@@ -48,6 +49,10 @@ __host__ __device__ inline size_t stash_floats_per_head(int T, int dk, int dv) {
 
 // Host launchers; return cudaSuccess or the launch error. Shapes are validated by the caller.
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
+
+// One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
+bool head_kernel_applies(const VerifyArgs& a);
+cudaError_t launch_verify_head(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
 
 }  // namespace gdn

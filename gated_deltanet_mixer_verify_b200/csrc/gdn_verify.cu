@@ -551,6 +551,7 @@ cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
+    if (head_kernel_applies(a)) return launch_verify_head(a, stream);
     switch (a.dk) {
         case 16: return launch_verify_dk<16>(a, stream);
         case 32: return launch_verify_dk<32>(a, stream);

@@ -73,7 +73,7 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /*
  * Problem description shared by all calls. Sizes supported by this build:
- *   B in 1..65535, H_v a multiple of H_k, H_v <= 65535,
+ *   B in 0..65535, H_v a multiple of H_k, H_v <= 65535, B * H_v <= 2^24,
  *   d_k in {16, 32, 64, 128, 256}, d_v in 1..4096,
  *   verify: T in 1..16; decode: T == 1; prefill: T >= 1, chunk == 64, d_k == d_v == 128.
  */

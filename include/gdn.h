@@ -69,12 +69,14 @@ typedef enum {
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Bits the kernels OR into *status_word. */
-#define GDN_STATUS_BAD_ACCEPT 1
+#define GDN_STATUS_BAD_ACCEPT 1     /* an accept_len[b] was outside 0..T: nothing committed for b */
+#define GDN_STATUS_WAIT_TIMEOUT 2   /* a bounded wait for an asynchronous copy ran out: the
+                                       affected heads were not written */
 
 /*
  * Problem description shared by all calls. Sizes supported by this build:
  *   B in 0..65535, H_v a multiple of H_k, H_v <= 65535, B * H_v <= 2^24,
- *   d_k in {16, 32, 64, 128, 256}, d_v in 1..4096,
+ *   d_k in {16, 32, 64, 128}, d_v in 1..4096,
  *   verify: T in 1..16; decode: T == 1; prefill: T >= 1, chunk == 64, d_k == d_v == 128.
  */
 typedef struct {

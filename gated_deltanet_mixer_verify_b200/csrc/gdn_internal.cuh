@@ -52,6 +52,10 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);
+
+// Tensor-core form (d_k = d_v = 128, T <= 8, at least one (sequence, head) per SM).
+bool tc_kernel_applies(const VerifyArgs& a, int num_sms);
+cudaError_t launch_verify_tc(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_verify_head(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
 

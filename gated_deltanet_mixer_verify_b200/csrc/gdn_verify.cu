@@ -551,6 +551,11 @@ cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
+    int dev = 0, nsm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);
     if (head_kernel_applies(a)) return launch_verify_head(a, stream);
     switch (a.dk) {
         case 16: return launch_verify_dk<16>(a, stream);

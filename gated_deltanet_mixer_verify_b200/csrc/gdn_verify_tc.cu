@@ -1,0 +1,452 @@
+// gdn_verify_tc.cu -- tensor-core form of the verify mixer for d_k = d_v = 128, T <= 8.
+//
+// Same block-form math as gdn_verify.cu (dots against the block's initial state, a T x T
+// unit-triangular solve, folded commit keys). The 2T dots per state row are a dense
+// contraction, P = S_0 [Khat; Qhat]^T (128 x 128 times 128 x 2T), so they run on the 5th-
+// generation tensor cores (tcgen05.mma, kind::tf32, fp32 accumulator in tensor memory) in
+// three passes, S_hi B_hi + S_hi B_lo + S_lo B_hi, where x_hi is x with its low 13 mantissa
+// bits cleared and x_lo = x - x_hi: this keeps the products accurate to about 2^-20 of fp32
+// (a single tf32 pass would be ~2^-11). The CUDA cores only split the state, run the small
+// per-head algebra, form outputs and write the committed rows.
+//
+// Shared memory holds the raw fp32 state tile (TMA, 128-byte swizzle): a kind::tf32 MMA
+// reads a 32-bit container as its truncated tf32 value, so that tile serves directly as S_hi.
+// S_lo = S - S_hi is formed by the threads and stored in tensor memory, where the third pass
+// takes its A operand. That keeps a CTA at ~100 KB of shared memory and 160 tensor-memory
+// columns, so two CTAs (16 warps) share an SM and overlap one head's copies and algebra with
+// the other's MMAs and commit. One CTA per (sequence, head).
+// Every mbarrier wait is bounded; a timeout sets GDN_STATUS_WAIT_TIMEOUT, suppresses the
+// CTA's global writes, drains its copy and MMAs (bounded) and frees its tensor memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn_device.cuh"
+#include "gdn_internal.cuh"
+#include "gdn_tc.cuh"
+
+namespace gdn {
+namespace {
+using namespace dev;
+
+constexpr int kThreads = 256;
+constexpr int DK = 128;
+constexpr int DV = 128;
+constexpr int TM = 8;                  // block length bound (N = 2 TM = 16)
+constexpr int NB = 2 * TM;             // rows of the B operand: khat_0..7, qhat_0..7
+constexpr uint32_t kTileBytes = DV * DK * 4;
+constexpr uint32_t kMaxPolls = 1u << 24;
+
+struct __align__(1024) TcSmem {
+    float S[DV * DK];        // raw fp32 state tile, SW128 K-major (4 blocks of [128 rows][32])
+    float Bh[NB * DK];       // [khat; qhat] high parts, SW128 K-major (4 blocks of [16][32])
+    float Bl[NB * DK];       // low parts
+    float KQ[NB][DK];        // khat, qhat in plain fp32 (Gram, Keff, stash)
+    float Keff[TM][DK];
+    float2 X2[DV][TM];       // (x_s, x_s) per state row: ready-made operands of the packed FMAs
+    float Gram[NB][TM];
+    float G[TM], Beta[TM], D[TM];
+    float A[TM][TM], Cq[TM][TM], Tm[TM][TM], Mo[TM][TM], E[TM][TM];
+    float DL;
+    int L;
+    int fail;                // a bounded wait ran out
+    uint32_t tmem_d;         // 32 columns: the dots, 128 lanes x 16
+    uint32_t tmem_a;         // 128 columns: S_lo as the A operand of the third pass
+    uint64_t full;
+    uint64_t mma_done;
+};
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Committed rows for a compile-time number LL of accepted tokens: S_L = d S_0 + sum_{s<LL}
+// x_s Keff_s (LL = 0: S_0 unchanged). One warp per 16 rows, a lane per 16-byte column chunk.
+template <int LL>
+__device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int warp, int lane, float dl) {
+    const int chunk = lane;   // columns 4*chunk .. +3
+    const int kb = chunk >> 3, c = chunk & 7;
+    float4 ke[LL > 0 ? LL : 1];
+#pragma unroll
+    for (int s = 0; s < LL; ++s) ke[s] = *reinterpret_cast<const float4*>(&sm.Keff[s][4 * chunk]);
+    const float2 dl2 = make_float2(dl, dl);
+#pragma unroll 4
+    for (int i = 0; i < DV / 8; ++i) {
+        const int row = warp + 8 * i;
+        const float4 sv =
+            *reinterpret_cast<const float4*>(&sm.S[(kb * DV * 128 + row * 128 + ((c ^ (row & 7)) << 4)) / 4]);
+        float2 r0 = make_float2(sv.x, sv.y), r1 = make_float2(sv.z, sv.w);
+        if (LL > 0) {
+            r0 = __fmul2_rn(r0, dl2);
+            r1 = __fmul2_rn(r1, dl2);
+#pragma unroll
+            for (int s = 0; s < LL; s += 2) {
+                const float4 xp = *reinterpret_cast<const float4*>(&sm.X2[row][s]);
+                const float2 xa = make_float2(xp.x, xp.y);
+                r0 = __ffma2_rn(xa, make_float2(ke[s].x, ke[s].y), r0);
+                r1 = __ffma2_rn(xa, make_float2(ke[s].z, ke[s].w), r1);
+                if (s + 1 < LL) {
+                    const float2 xb = make_float2(xp.z, xp.w);
+                    r0 = __ffma2_rn(xb, make_float2(ke[s + 1].x, ke[s + 1].y), r0);
+                    r1 = __ffma2_rn(xb, make_float2(ke[s + 1].z, ke[s + 1].w), r1);
+                }
+            }
+        }
+        __stcs(reinterpret_cast<float4*>(dst + (size_t)row * DK) + chunk, make_float4(r0.x, r0.y, r1.x, r1.y));
+    }
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(kThreads, 2)
+    gdn_verify_tc_kernel(const __grid_constant__ CUtensorMap smap, const VerifyArgs p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw);
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int T = p.T;
+    const int item = blockIdx.x;
+    const int h = item % p.Hv;
+    const int b = item / p.Hv;
+    const int g = h / (p.Hv / p.Hk);
+    const size_t head = (size_t)item;
+    const size_t tok_stride = (size_t)p.Hv * DV;               // between tokens in v and o
+    const size_t vo_base = ((size_t)b * T * p.Hv + h) * DV;    // token 0, row 0 of this head
+
+    if ((smem_u32(smem_raw) & 1023u) != 0) {   // the swizzled tiles need 1024-byte alignment
+        if (tid == 0 && p.status_word) atomicOr(p.status_word, kStatusWaitTimeout);
+        return;
+    }
+
+    // 0. Request the head's state; allocate tensor memory.
+    if (tid == 0) {
+        mbar_init(&sm.full, 1);
+        mbar_init(&sm.mma_done, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&sm.full, kTileBytes);
+        for (int kb = 0; kb < 4; ++kb) tc::tma_load_2d(&sm.S[kb * DV * 32], &smap, kb * 32, item * DV, &sm.full);
+        sm.fail = 0;
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.tmem_d, 32);
+        tc::tmem_alloc(&sm.tmem_a, 128);
+        tc::tmem_relinquish();
+    }
+
+    // Per-row v_t, fetched early (rows 0..127 belong to threads 0..127).
+    float vrow[TM];
+#pragma unroll
+    for (int t = 0; t < TM; ++t)
+        vrow[t] = (tid < DV && t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + tid) : 0.f;
+
+    // 1a. khat_t, qhat_t: 16 lanes per vector, 8 columns per lane; plain copy + split tiles.
+    {
+        const int c16 = tid & 15;
+        const int n = tid >> 4;              // 0..15 = NB rows
+        const bool isq = n >= TM;
+        const int t = isq ? n - TM : n;
+        const bool live = t < T;
+        float x[8];
+        if (live) {
+            ld8<InT>(isq ? p.q : p.k, (((size_t)b * T + t) * p.Hk + g) * DK + 8 * c16, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+        ss = group_sum<16>(ss);
+        const float inv = live ? (isq ? p.scale : 1.f) / sqrtf(ss + p.l2_eps) : 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float4 y, hi, lo;
+            y = make_float4(x[4 * half] * inv, x[4 * half + 1] * inv, x[4 * half + 2] * inv, x[4 * half + 3] * inv);
+            hi = make_float4(tc::tf32_hi(y.x), tc::tf32_hi(y.y), tc::tf32_hi(y.z), tc::tf32_hi(y.w));
+            lo = make_float4(y.x - hi.x, y.y - hi.y, y.z - hi.z, y.w - hi.w);
+            const uint32_t o = tc::sw128_offset(n, 8 * c16 + 4 * half, NB) / 4;
+            *reinterpret_cast<float4*>(&sm.Bh[o]) = hi;
+            *reinterpret_cast<float4*>(&sm.Bl[o]) = lo;
+            *reinterpret_cast<float4*>(&sm.KQ[n][8 * c16 + 4 * half]) = y;
+        }
+    }
+
+    // 1b. Gates and the inclusive prefix sum of log-decays (warp 0, lane t = token t).
+    if (warp == 0) {
+        float gl = 0.f, be = 0.f;
+        if (lane < T) {
+            const size_t gi = ((size_t)b * T + lane) * p.Hv + h;
+            gl = -expf(p.A_log[h]) * softplus_f(ld_in<InT>(p.a, gi) + p.dt_bias[h]);
+            be = 1.f / (1.f + expf(-ld_in<InT>(p.b, gi)));
+        }
+        float Gs = gl;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(kFull, Gs, off);
+            if (lane >= off) Gs += y;
+        }
+        if (lane < TM) {
+            sm.G[lane] = Gs;
+            sm.Beta[lane] = be;
+            sm.D[lane] = (lane < T) ? expf(Gs) : 0.f;
+        }
+        if (lane == 0) {
+            int L;
+            if (p.always_commit) {
+                L = T;
+            } else if (p.accept_len) {
+                L = p.accept_len[b];
+                if (L < 0 || L > T) {
+                    if (p.status_word && h == 0) atomicOr(p.status_word, kStatusBadAccept);
+                    L = -1;
+                }
+            } else {
+                L = -2;
+            }
+            sm.L = L;
+        }
+    }
+    tc::fence_proxy_async_smem();   // the tensor core will read the B tiles written above
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem_d = sm.tmem_d, tmem_a = sm.tmem_a;
+
+    if (warp >= 4) {
+        // 2s. Warps 4..7: S_lo = S - trunc_tf32(S) into tensor memory (warp w owns lanes
+        // 32 (w - 4) .. +31, i.e. those state rows, all 128 columns), then one thread issues
+        // the three tf32 passes: S (smem) B_hi + S (smem) B_lo + S_lo (tmem) B_hi.
+        const int q4 = warp - 4;
+        const int row = 32 * q4 + lane;
+        if (!mbar_wait_bounded(&sm.full, 0, kMaxPolls)) sm.fail = 1;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            float v[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 x = *reinterpret_cast<const float4*>(
+                    &sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
+                v[4 * q + 0] = x.x - tc::tf32_hi(x.x);
+                v[4 * q + 1] = x.y - tc::tf32_hi(x.y);
+                v[4 * q + 2] = x.z - tc::tf32_hi(x.z);
+                v[4 * q + 3] = x.w - tc::tf32_hi(x.w);
+            }
+            tc::tmem_st32(tmem_a + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
+        }
+        tc::fence_before_sync();
+        named_sync(2, 128);
+        tc::fence_after_sync();
+        if (tid == 128 && !sm.fail) {
+            const uint32_t id = tc::idesc_tf32(DV, NB);
+            const uint32_t as = smem_u32(sm.S);
+            const uint32_t bh = smem_u32(sm.Bh), bl = smem_u32(sm.Bl);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_tf32_ss(tmem_d, tc::desc_kmajor_sw128(as + kb * DV * 128 + ks * 32),
+                                    tc::desc_kmajor_sw128(bh + kb * NB * 128 + ks * 32), id, kb + ks > 0);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_tf32_ss(tmem_d, tc::desc_kmajor_sw128(as + kb * DV * 128 + ks * 32),
+                                    tc::desc_kmajor_sw128(bl + kb * NB * 128 + ks * 32), id, true);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_tf32_ts(tmem_d, tmem_a + kb * 32 + ks * 8,
+                                    tc::desc_kmajor_sw128(bh + kb * NB * 128 + ks * 32), id, true);
+            tc::mma_commit(&sm.mma_done);
+        }
+    } else {
+        // 2a. Warps 0..3 meanwhile: Gram rows [Khat; Qhat] Khat^T (8 lanes per row, interleaved
+        // float4 columns, halving butterfly) ...
+        {
+            const int c8 = tid & 7;
+            const int n = tid >> 3;          // 0..15
+            float4 xr[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) xr[m] = *reinterpret_cast<const float4*>(&sm.KQ[n][4 * (c8 + 8 * m)]);
+            float part[TM];
+#pragma unroll
+            for (int s = 0; s < TM; ++s) {
+                float d = 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float4 y = *reinterpret_cast<const float4*>(&sm.KQ[s][4 * (c8 + 8 * m)]);
+                    d = fmaf(xr[m].x, y.x, d);
+                    d = fmaf(xr[m].y, y.y, d);
+                    d = fmaf(xr[m].z, y.z, d);
+                    d = fmaf(xr[m].w, y.w, d);
+                }
+                part[s] = d;
+            }
+            Halve<TM, 4>::run(part, c8);
+            sm.Gram[n][c8] = part[0];
+        }
+        named_sync(1, 128);
+        // ... the decayed coefficients, the triangular inverse, output and commit coefficients
+        // (warp 0) ...
+        if (warp == 0) {
+            for (int e = lane; e < TM * TM; e += 32) {
+                const int t = e / TM, s = e % TM;
+                const bool inq = t < T && s <= t;
+                const float dec = inq ? expf(sm.G[t] - sm.G[s]) : 0.f;
+                sm.A[t][s] = (inq && s < t) ? sm.Beta[t] * dec * sm.Gram[t][s] : 0.f;
+                sm.Cq[t][s] = inq ? dec * sm.Gram[TM + t][s] : 0.f;
+            }
+            __syncwarp();
+            if (lane < TM) {
+                const int s = lane;
+                float col[TM];
+#pragma unroll
+                for (int t = 0; t < TM; ++t) {
+                    float x = (t == s) ? 1.f : 0.f;
+#pragma unroll
+                    for (int m = 0; m < t; ++m) x = fmaf(-sm.A[t][m], col[m], x);
+                    col[t] = (t >= s) ? x : 0.f;
+                    sm.Tm[t][s] = col[t];
+                }
+            }
+            __syncwarp();
+            const int L = sm.L;
+            for (int e = lane; e < TM * TM; e += 32) {
+                const int t = e / TM, s = e % TM;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < TM; ++m)
+                    if (m >= s && m <= t) acc = fmaf(sm.Cq[t][m], sm.Tm[m][s], acc);
+                sm.Mo[t][s] = (s <= t) ? acc : 0.f;
+                sm.E[t][s] = (L > 0 && t < L && s <= t) ? expf(sm.G[L - 1] - sm.G[t]) * sm.Tm[t][s] : 0.f;
+            }
+            if (lane == 0) sm.DL = (L > 0) ? sm.D[L - 1] : 1.f;
+        }
+        named_sync(1, 128);
+        // ... and Keff_s = sum_t E[t][s] khat_t (warps 0..3, column j = tid, 8 entries each).
+        if (sm.L > 0) {
+#pragma unroll
+            for (int s = 0; s < TM; ++s) {
+                float acc = 0.f;
+#pragma unroll
+                for (int t = 0; t < TM; ++t) acc = fmaf(sm.E[t][s], sm.KQ[t][tid], acc);
+                sm.Keff[s][tid] = acc;
+            }
+        }
+    }
+    __syncthreads();
+    const int L = sm.L;
+    bool ok = !sm.fail;
+
+    // 3. Rows 0..127 (threads 0..127, one row each): the dots from tensor memory, x_s, the
+    // outputs and (two-phase) the stash; warps 4..7 write the stash's keys and decays.
+    if (ok && !mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls)) ok = false;
+    tc::fence_after_sync();
+    if (warp < 4) {
+        float dots[16];
+        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * warp) << 16), dots);
+        const int row = tid;
+        float xs[TM];
+#pragma unroll
+        for (int s = 0; s < TM; ++s) xs[s] = sm.Beta[s] * (vrow[s] - sm.D[s] * dots[s]);
+#pragma unroll
+        for (int s = 0; s < TM; s += 2)
+            *reinterpret_cast<float4*>(&sm.X2[row][s]) = make_float4(xs[s], xs[s], xs[s + 1], xs[s + 1]);
+        if (ok) {
+            OutT* op = reinterpret_cast<OutT*>(p.o);
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                if (t < T) {
+                    float ov = sm.D[t] * dots[TM + t];
+#pragma unroll
+                    for (int s = 0; s <= t; ++s) ov = fmaf(sm.Mo[t][s], xs[s], ov);
+                    st_out<OutT>(op, vo_base + t * tok_stride + row, ov);
+                }
+            }
+            if (p.stash) {
+                float* st = p.stash + head * stash_floats_per_head(T, DK, DV);
+                const size_t off_u = (size_t)T * DK + (((size_t)T + 3) & ~size_t(3));
+#pragma unroll
+                for (int t = 0; t < TM; ++t) {
+                    if (t < T) {
+                        float u = 0.f;
+#pragma unroll
+                        for (int s = 0; s <= t; ++s) u = fmaf(sm.Tm[t][s], xs[s], u);
+                        st[off_u + (size_t)t * DV + row] = u;
+                    }
+                }
+            }
+        }
+    } else if (p.stash && ok) {
+        float* st = p.stash + head * stash_floats_per_head(T, DK, DV);
+        for (int e = tid - 128; e < T * DK; e += 128) st[e] = sm.KQ[e / DK][e % DK];
+        if (tid - 128 < T) st[(size_t)T * DK + (tid - 128)] = sm.G[tid - 128];
+    }
+    tc::fence_before_sync();
+    ok = !__syncthreads_or(!ok);
+    if (!ok && tid == 0 && p.status_word) atomicOr(p.status_word, kStatusWaitTimeout);
+
+    // 4. Commit at L (rollback / bad L: the initial state, skipped when in place).
+    if (ok && (L != -2) && !(L <= 0 && p.state_out == p.state_in)) {
+        float* dst = p.state_out + head * (size_t)DV * DK;
+        const float dl = sm.DL;
+        switch (L > 0 ? L : 0) {
+            case 1: commit_rows<1>(sm, dst, warp, lane, dl); break;
+            case 2: commit_rows<2>(sm, dst, warp, lane, dl); break;
+            case 3: commit_rows<3>(sm, dst, warp, lane, dl); break;
+            case 4: commit_rows<4>(sm, dst, warp, lane, dl); break;
+            case 5: commit_rows<5>(sm, dst, warp, lane, dl); break;
+            case 6: commit_rows<6>(sm, dst, warp, lane, dl); break;
+            case 7: commit_rows<7>(sm, dst, warp, lane, dl); break;
+            case 8: commit_rows<8>(sm, dst, warp, lane, dl); break;
+            default: commit_rows<0>(sm, dst, warp, lane, dl); break;
+        }
+    }
+
+    // Drain after a timeout (bounded), then free the tensor memory (always).
+    if (!ok && tid == 0) {
+        mbar_wait_bounded(&sm.full, 0, kMaxPolls);
+        if (!sm.fail) mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tmem_dealloc(tmem_a, 128);
+        tc::tmem_dealloc(tmem_d, 32);
+    }
+}
+
+template <typename InT, typename OutT>
+cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
+    constexpr size_t smem = sizeof(TcSmem);
+    static bool configured = false;   // per process; the attribute is per function
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    CUtensorMap map;
+    cudaError_t e = tc::encode_tmap_f32_sw128(&map, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
+    if (e != cudaSuccess) return e;
+    gdn_verify_tc_kernel<InT, OutT><<<a.B * a.Hv, kThreads, smem, stream>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_kernel_applies(const VerifyArgs& a, int num_sms) {
+    // Single-token decode stays on the CUDA-core head kernel (measured faster there).
+    return a.dk == DK && a.dv == DV && a.T >= 2 && a.T <= TM && (long long)a.B * a.Hv >= num_sms;
+}
+
+cudaError_t launch_verify_tc(const VerifyArgs& a, cudaStream_t stream) {
+    if (a.in_bf16)
+        return a.out_bf16 ? launch_tc_t<__nv_bfloat16, __nv_bfloat16>(a, stream)
+                          : launch_tc_t<__nv_bfloat16, float>(a, stream);
+    return a.out_bf16 ? launch_tc_t<float, __nv_bfloat16>(a, stream) : launch_tc_t<float, float>(a, stream);
+}
+
+}  // namespace gdn

@@ -40,8 +40,8 @@ constexpr uint32_t kMaxPolls = 1u << 24;
 
 struct __align__(1024) TcSmem {
     float S[DV * DK];        // raw fp32 state tile, SW128 K-major (4 blocks of [128 rows][32])
-    float Bh[NB * DK];       // [khat; qhat] high parts, SW128 K-major (4 blocks of [16][32])
-    float Bl[NB * DK];       // low parts
+    float B2[2 * NB * DK];   // rows 0..15: [khat; qhat] high parts, rows 16..31: low parts;
+                             // SW128 K-major (4 blocks of [32 rows][32])
     float KQ[NB][DK];        // khat, qhat in plain fp32 (Gram, Keff, stash)
     float Keff[TM][DK];
     float2 X2[DV][TM];       // (x_s, x_s) per state row: ready-made operands of the packed FMAs
@@ -165,9 +165,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             y = make_float4(x[4 * half] * inv, x[4 * half + 1] * inv, x[4 * half + 2] * inv, x[4 * half + 3] * inv);
             hi = make_float4(tc::tf32_hi(y.x), tc::tf32_hi(y.y), tc::tf32_hi(y.z), tc::tf32_hi(y.w));
             lo = make_float4(y.x - hi.x, y.y - hi.y, y.z - hi.z, y.w - hi.w);
-            const uint32_t o = tc::sw128_offset(n, 8 * c16 + 4 * half, NB) / 4;
-            *reinterpret_cast<float4*>(&sm.Bh[o]) = hi;
-            *reinterpret_cast<float4*>(&sm.Bl[o]) = lo;
+            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(n, 8 * c16 + 4 * half, 2 * NB) / 4]) = hi;
+            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(NB + n, 8 * c16 + 4 * half, 2 * NB) / 4]) = lo;
             *reinterpret_cast<float4*>(&sm.KQ[n][8 * c16 + 4 * half]) = y;
         }
     }
@@ -238,27 +237,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         named_sync(2, 128);
         tc::fence_after_sync();
         if (tid == 128 && !sm.fail) {
-            const uint32_t id = tc::idesc_tf32(DV, NB);
+            // Columns 0..15 accumulate S B_hi + S_lo B_hi, columns 16..31 S B_lo.
+            const uint32_t id32 = tc::idesc_tf32(DV, 2 * NB), id16 = tc::idesc_tf32(DV, NB);
             const uint32_t as = smem_u32(sm.S);
-            const uint32_t bh = smem_u32(sm.Bh), bl = smem_u32(sm.Bl);
+            const uint32_t bb = smem_u32(sm.B2);
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_tf32_ss(tmem_d, tc::desc_kmajor_sw128(as + kb * DV * 128 + ks * 32),
-                                    tc::desc_kmajor_sw128(bh + kb * NB * 128 + ks * 32), id, kb + ks > 0);
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_tf32_ss(tmem_d, tc::desc_kmajor_sw128(as + kb * DV * 128 + ks * 32),
-                                    tc::desc_kmajor_sw128(bl + kb * NB * 128 + ks * 32), id, true);
+                                    tc::desc_kmajor_sw128(bb + kb * 2 * NB * 128 + ks * 32), id32, kb + ks > 0);
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_tf32_ts(tmem_d, tmem_a + kb * 32 + ks * 8,
-                                    tc::desc_kmajor_sw128(bh + kb * NB * 128 + ks * 32), id, true);
+                                    tc::desc_kmajor_sw128(bb + kb * 2 * NB * 128 + ks * 32), id16, true);
             tc::mma_commit(&sm.mma_done);
         }
     } else {
@@ -345,8 +339,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok && !mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls)) ok = false;
     tc::fence_after_sync();
     if (warp < 4) {
-        float dots[16];
+        float dots[16], dlo[16];
         tc::tmem_ld16(tmem_d + ((uint32_t)(32 * warp) << 16), dots);
+        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * warp) << 16) + 16, dlo);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dots[i] += dlo[i];
         const int row = tid;
         float xs[TM];
 #pragma unroll

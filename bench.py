@@ -34,7 +34,13 @@ from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload  # noq
 METRIC = "GDN verify/decode HBM GB/s (frac of B200 peak), token·heads/s; prefill tok/s"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+# Sources of the dominant kernels; a committed ncu traffic figure is only reported while
+# these are unchanged.
 KERNEL_SOURCES = ["gated_deltanet_mixer_verify_b200/csrc/gdn_verify.cu",
+                  "gated_deltanet_mixer_verify_b200/csrc/gdn_verify_tc.cu",
+                  "gated_deltanet_mixer_verify_b200/csrc/gdn_verify_head.cu",
+                  "gated_deltanet_mixer_verify_b200/csrc/gdn_tc.cuh",
+                  "gated_deltanet_mixer_verify_b200/csrc/gdn_device.cuh",
                   "gated_deltanet_mixer_verify_b200/csrc/gdn_internal.cuh"]
 
 

@@ -16,9 +16,6 @@ int check_prefill_shape(const gdn_shape* s, int chunk);
 // Scratch bytes the prefill needs (0 when it needs none).
 size_t prefill_workspace_bytes(int B, int T, int Hv, int dk, int dv, int chunk);
 
-// The CUDA-core scan: the verify kernel taken over the whole prompt in 16-token blocks,
-// with each CTA's state rows kept in registers from block to block.
-cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t stream);
 
 cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);

@@ -534,21 +534,7 @@ cudaError_t launch_commit_dk(const CommitArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int DK, typename InT, typename OutT>
-cudaError_t launch_scan_t(const VerifyArgs& a, cudaStream_t stream) {
-    return launch_verify_t<DK, 16, InT, OutT>(a, stream);
-}
-
 }  // namespace
-
-cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t stream) {
-    if (a.dk != 128) return cudaErrorInvalidValue;
-    if (a.in_bf16)
-        return a.out_bf16 ? launch_scan_t<128, __nv_bfloat16, __nv_bfloat16>(a, stream)
-                          : launch_scan_t<128, __nv_bfloat16, float>(a, stream);
-    return a.out_bf16 ? launch_scan_t<128, float, __nv_bfloat16>(a, stream)
-                      : launch_scan_t<128, float, float>(a, stream);
-}
 
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
     int dev = 0, nsm = 0;

@@ -251,6 +251,46 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* 
                     who);
 }
 
+gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,
+                                     const void* v, const void* a, const void* b, const float* A_log,
+                                     const float* dt_bias, const float* state_in, float* state_out, void* o,
+                                     void* stream) {
+    const char* who = "gdn_chunk_prefill_noalloc";
+    if (!shape) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
+    gdn_status st = check_shape(shape, 1 << 30, who);
+    if (st != GDN_OK) return st;
+    if (gdn::check_prefill_shape(shape, chunk) != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: only chunk 64 with d_k = d_v = 128 is built", who);
+    if (shape->B == 0) return ok();
+    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k,
+                                                     shape->d_v, chunk);
+    if (need > gdn::kNoAllocScratchBytes)
+        return fail(GDN_ERR_UNSUPPORTED,
+                    "%s: this shape needs %zu bytes of scratch, the fixed scratch holds %zu; "
+                    "use gdn_chunk_prefill with a workspace",
+                    who, need, gdn::kNoAllocScratchBytes);
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    REQUIRE_PTR(state_out, who);
+    REQUIRE_PTR(o, who);
+    if (state_in) {
+        REQUIRE_PTR(state_in, who);
+        if (!overlap_ok(state_in, state_out, state_bytes(shape)))
+            return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
+    }
+    gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
+    x.state_in = state_in;
+    x.state_out = state_out;
+    x.o = o;
+    x.always_commit = 1;
+    return launched(gdn::launch_prefill_noalloc(x, chunk, static_cast<cudaStream_t>(stream)), who);
+}
+
 const char* gdn_status_string(gdn_status status) {
     switch (status) {
         case GDN_OK: return "GDN_OK";

@@ -29,6 +29,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "gdn_device.cuh"
 #include "gdn_internal.cuh"
 #include "gdn_prefill.cuh"
@@ -251,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------- scan kernel
+
 
 struct __align__(1024) ScanSmem {
     float KQ[2 * kC * DK];       // [khat; qhat] rows of the current chunk, SW128 K-major
@@ -558,7 +561,43 @@ cudaError_t launch_tc_prefill(const VerifyArgs& a, void* workspace, cudaStream_t
     return cudaGetLastError();
 }
 
+// Fixed scratch for gdn_chunk_prefill_noalloc. It is a module-scope device array, so every
+// GPU that loads this library holds it (kNoAllocScratchBytes) until the process exits, and
+// every call of that entry point on one GPU reuses the same bytes.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's name
+// is only a host-side stand-in, so the address is asked of the runtime, once per device (with
+// that device current), and cached.
+cudaError_t noalloc_scratch_address(void** out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
 }  // namespace
+
+cudaError_t launch_prefill_noalloc(const VerifyArgs& a, int chunk, cudaStream_t stream) {
+    // Nothing in the scratch has to start at zero: the prep kernel writes every workspace
+    // element the scan kernel reads, on the same stream, before the scan reads it.
+    void* ws = nullptr;
+    cudaError_t e = noalloc_scratch_address(&ws);
+    if (e != cudaSuccess) return e;
+    return launch_prefill(a, chunk, ws, kNoAllocScratchBytes, stream);
+}
 
 int check_prefill_shape(const gdn_shape* s, int chunk) {
     if (!s) return -1;

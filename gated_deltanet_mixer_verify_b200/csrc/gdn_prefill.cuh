@@ -20,4 +20,10 @@ size_t prefill_workspace_bytes(int B, int T, int Hv, int dk, int dv, int chunk);
 cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+// Size of the fixed device scratch behind gdn_chunk_prefill_noalloc (include/gdn.h).
+constexpr size_t kNoAllocScratchBytes = GDN_NOALLOC_SCRATCH_BYTES;
+
+// The prefill with its workspace in that fixed scratch; the caller checks the size.
+cudaError_t launch_prefill_noalloc(const VerifyArgs& a, int chunk, cudaStream_t stream);
+
 }  // namespace gdn

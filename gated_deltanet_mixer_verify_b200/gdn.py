@@ -60,7 +60,9 @@ def _load():
     lib.gdn_commit.argtypes = [S] + [_VP] * 5
     lib.gdn_decode_step.argtypes = [S] + [_VP] * 10
     lib.gdn_chunk_prefill.argtypes = ([S, ctypes.c_int32] + [_VP] * 11 + [ctypes.c_size_t, _VP])
-    for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill"):
+    lib.gdn_chunk_prefill_noalloc.argtypes = [S, ctypes.c_int32] + [_VP] * 11
+    for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill",
+               "gdn_chunk_prefill_noalloc"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -201,4 +203,29 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, 
                                      _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state_in),
                                      _ptr(state_out), _ptr(o), _ptr(workspace), wbytes,
                                      _stream(stream)))
+    return o, state_out
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, o=None,
+                          chunk=64, l2_eps=1e-6, scale=1.0, status_word=None,
+                          out_dtype=torch.float32, stream=None):
+    """chunk_prefill without a workspace, for callers that cannot allocate device memory.
+
+    The library's fixed device scratch (NOALLOC_SCRATCH_BYTES per GPU) is used instead; shapes
+    that need more raise GdnError. Calls that overlap on the GPU share that scratch and race.
+    ``o`` and ``state_out`` are the caller's; they are only created here when omitted."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    B, T, H_k, d_k = k.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    if state_out is None:
+        state_out = torch.empty((B, H_v, d_v, d_k), dtype=torch.float32, device=v.device)
+    _check(_load().gdn_chunk_prefill_noalloc(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                                             _ptr(state_in), _ptr(state_out), _ptr(o),
+                                             _stream(stream)))
     return o, state_out

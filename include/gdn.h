@@ -156,6 +156,39 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
                              const float* state_in, float* state_out, void* o,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the fixed device scratch behind gdn_chunk_prefill_noalloc: 64 MiB. */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * gdn_chunk_prefill_noalloc -- gdn_chunk_prefill for callers that cannot allocate device
+ * memory. (The source pages have no counterpart; this is a convenience of this library.)
+ *
+ * Some callers cannot hand the prefill a workspace: an engine whose memory manager reserved
+ * all device memory at start-up and will not give out more, or a hot path that must not
+ * enter the CUDA allocator because cudaMalloc / cudaFree can synchronise the device and stall
+ * every stream. This entry point takes the same arguments as gdn_chunk_prefill minus the
+ * workspace, and uses a fixed scratch array that is part of the library's device code instead:
+ *   - The scratch is GDN_NOALLOC_SCRATCH_BYTES. Every GPU that loads the library keeps it
+ *     allocated until the process exits, whether or not this entry point is called.
+ *   - Shapes whose workspace (gdn_chunk_prefill_workspace_bytes) exceeds it are rejected with
+ *     GDN_ERR_UNSUPPORTED and a gdn_last_error() message giving both sizes; with d = 128 and
+ *     chunk 64 each (sequence, value head, 64-token chunk) needs 49,728 bytes, e.g. up to 28
+ *     chunks (1,792 tokens) for B = 1 and H_v = 48.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - All calls on one GPU share the same scratch and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each call writes every element it later reads),
+ *     but calls that may overlap on the GPU -- on different streams without ordering between
+ *     them -- race on the scratch and can corrupt each other's results. Order them.
+ *   - The first call on a device looks up the scratch's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ */
+gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk,
+                                     const void* q, const void* k, const void* v,
+                                     const void* a, const void* b,
+                                     const float* A_log, const float* dt_bias,
+                                     const float* state_in, float* state_out, void* o,
+                                     void* stream);
+
 /* Bytes of stash gdn_verify_step writes for this shape (0 for an invalid shape). */
 size_t gdn_stash_bytes(const gdn_shape* shape);
 

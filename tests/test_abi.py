@@ -87,6 +87,10 @@ def test_host_validation_rejects_before_launch(gdn):
     assert lib.gdn_chunk_prefill(ctypes.byref(sh), 32, *([0x10000] * 11), 0, None) == UNSUP
     sh = ok_shape(T=4096, d_k=64, d_v=64)
     assert lib.gdn_chunk_prefill(ctypes.byref(sh), 64, *([0x10000] * 11), 0, None) == UNSUP
+    # the no-allocation prefill refuses shapes larger than its fixed scratch, before any launch
+    sh = ok_shape(B=1, T=4096)
+    assert lib.gdn_chunk_prefill_noalloc(ctypes.byref(sh), 64, *([0x10000] * 10), None) == UNSUP
+    assert "fixed scratch" in lib.gdn_last_error().decode()
 
 
 def test_empty_batch_is_a_no_op(gdn):

@@ -241,10 +241,14 @@ class SingleSeq:
 
 
 class Prefill:
+    tokens = 0   # prompt length override (0: the workload's)
+
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
         self.gdn = gdn
         self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
+        if Prefill.tokens:
+            self.w = workload(name, seed=self.w.seed, T=Prefill.tokens)
         x = make_inputs(self.w)
         self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
         w = self.w
@@ -265,7 +269,9 @@ class Prefill:
                                None, self.state, self.o, self.w.chunk, self.ws)
 
     def config(self):
-        return workload_config(self.w.name)
+        c = workload_config(self.w.name)
+        c["T"] = self.w.T
+        return c
 
 
 WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
@@ -370,6 +376,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_verify")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="prefill only: prompt length override (default 32768), for profiling a "
+                         "smaller case")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -392,6 +401,7 @@ def main():
         if world > 1:
             dist.barrier()
 
+    Prefill.tokens = args.tokens
     wl = WORKLOADS[args.workload](args.workload, rank, dev)
     stream = torch.cuda.current_stream(dev)
 

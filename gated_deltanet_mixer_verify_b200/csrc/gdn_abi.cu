@@ -204,7 +204,7 @@ size_t gdn_stash_bytes(const gdn_shape* shape) {
 
 size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk) {
     if (gdn::check_prefill_shape(shape, chunk) != 0) return 0;
-    return gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k, shape->d_v, chunk);
+    return gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k, shape->d_v, chunk);
 }
 
 gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,
@@ -233,7 +233,7 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* 
         if (!overlap_ok(state_in, state_out, state_bytes(shape)))
             return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
     }
-    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k,
+    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k,
                                                      shape->d_v, chunk);
     if (need > 0) {
         if (!workspace || workspace_bytes < need)
@@ -262,7 +262,7 @@ gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk, cons
     if (gdn::check_prefill_shape(shape, chunk) != 0)
         return fail(GDN_ERR_UNSUPPORTED, "%s: only chunk 64 with d_k = d_v = 128 is built", who);
     if (shape->B == 0) return ok();
-    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_v, shape->d_k,
+    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k,
                                                      shape->d_v, chunk);
     if (need > gdn::kNoAllocScratchBytes)
         return fail(GDN_ERR_UNSUPPORTED,

@@ -14,7 +14,7 @@ namespace gdn {
 int check_prefill_shape(const gdn_shape* s, int chunk);
 
 // Scratch bytes the prefill needs (0 when it needs none).
-size_t prefill_workspace_bytes(int B, int T, int Hv, int dk, int dv, int chunk);
+size_t prefill_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk);
 
 
 cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size_t workspace_bytes,

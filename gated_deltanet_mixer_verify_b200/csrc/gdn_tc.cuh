@@ -120,6 +120,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Store 16 consecutive 32-bit columns of this thread's lane (no wait; see tmem_st_wait).
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+        : "memory");
+}
+
+// Wait for this thread's outstanding tcgen05.st.
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Store 32 consecutive 32-bit columns of this thread's lane, then wait for the store.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
@@ -147,6 +160,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 4-D tiled tensor copy global -> shared (coordinates innermost first; c0 * element size a
+// multiple of 16 bytes), completion counted on `bar`. Elements outside the tensor read as zero.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(d),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(b)
+        : "memory");
+}
+
+// x rounded to the nearest tf32 value (ties away from zero), in a 32-bit container whose low
+// 13 mantissa bits are zero, so that a kind::tf32 MMA multiplies it exactly.
+__device__ __forceinline__ float tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
 // tf32 value of x with the low 13 mantissa bits cleared (exactly representable in tf32). This
 // is also the value a kind::tf32 MMA uses when it reads x from a 32-bit container (the low
 // bits are ignored, not rounded).
@@ -159,6 +193,12 @@ __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__flo
 // looked up at run time, so the library does not link against libcuda).
 cudaError_t encode_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                                   uint32_t box_rows);
+
+// Encode a 4-D tensor map over a row-major [B][T][heads][d] array of fp32 or bf16 with a box of
+// `box_tokens` tokens of one head ([box_tokens][d] in shared memory, unswizzled). Tokens past T
+// read as zero. d * element size must be a multiple of 16 bytes and d <= 256.
+cudaError_t encode_tmap_tokens(CUtensorMap* map, const void* base, bool bf16, uint64_t d, uint64_t heads,
+                               uint64_t T, uint64_t B, uint32_t box_tokens);
 
 }  // namespace tc
 }  // namespace gdn

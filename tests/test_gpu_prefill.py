@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from gated_deltanet_mixer_verify_b200.inputs import as_f64, make_inputs, workload
-from gdn_helpers import TOL_PREFILL, rel_err, to_dev
+from gdn_helpers import TOL_BF16_OUT, TOL_PREFILL, rel_err, to_dev
 from oracle import gdn_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -57,3 +57,43 @@ def test_prefill_full_prompt_sampled_heads(gdn):
         o_ref, S_ref = orc.prefill(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"])
         assert rel_err(o[:, :, h:h + 1], o_ref) <= TOL_PREFILL, h
         assert rel_err(S[:, h:h + 1], S_ref) <= TOL_PREFILL, h
+
+
+def _oracle_prefill(x, with_state):
+    f = as_f64(x)
+    return orc.prefill(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"],
+                       f["S0"] if with_state else None)
+
+
+def test_prefill_long_gentle_decay_with_state(gdn):
+    # Mild gates: the state's running decay crosses 2^-32 every dozen chunks or so, so the
+    # kernel's lazy decay scalar and its occasional rescale of the stored state both run.
+    w = workload("prefill", T=2048, H_k=1, H_v=2, seed=77, state_std=0.05)
+    x = make_inputs(w, gates="gentle")
+    o_ref, S_ref = _oracle_prefill(x, True)
+    xd = to_dev(x)
+    o, S = run_gpu(gdn, xd, xd["S0"])
+    assert rel_err(o, o_ref) <= TOL_PREFILL and rel_err(S, S_ref) <= TOL_PREFILL
+
+
+def test_prefill_fp32_inputs_bf16_outputs(gdn):
+    w = workload("prefill", T=200, H_k=2, H_v=4, seed=78, in_dtype="f32", state_std=0.05)
+    x = make_inputs(w, gates="gentle")
+    o_ref, S_ref = _oracle_prefill(x, True)
+    xd = to_dev(x)
+    o, S = gdn.chunk_prefill(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["A_log"], xd["dt_bias"],
+                             xd["S0"], None, None, 64, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    assert rel_err(o, o_ref) <= TOL_BF16_OUT and rel_err(S, S_ref) <= TOL_PREFILL
+
+
+def test_prefill_batch_of_two_grouped_heads(gdn):
+    # Two sequences, two value heads per key head: each key head's normalised tile is written
+    # once and read by both of its value heads; a ragged last chunk (T % 64 = 3).
+    w = workload("prefill", B=2, T=131, H_k=2, H_v=4, seed=79, state_std=0.05)
+    x = make_inputs(w, gates="gentle")
+    o_ref, S_ref = _oracle_prefill(x, True)
+    xd = to_dev(x)
+    o, S = run_gpu(gdn, xd, xd["S0"])
+    assert rel_err(o, o_ref) <= TOL_PREFILL and rel_err(S, S_ref) <= TOL_PREFILL

@@ -71,6 +71,19 @@ __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error about 2^-22, subnormal
+// results flushed to zero).
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Named barrier `id` (1..15) over the first `nthreads` threads of the block (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 
 // Halving butterfly over the lanes of an aligned group (lane bits below 2*OFF). On return a

@@ -12,17 +12,19 @@
 //   O[i][t] = d_t R[i][t] + (X Mo^T)[i][t]
 //   S      <- d_C S + X Keff
 // Two kernels:
-//   gdn_prefill_prep_kernel, one CTA per (sequence, value head, chunk), all in parallel: the
-//     state-independent part. Normalised keys / queries and their Gram matrix (tensor cores);
+//   gdn_prefill_prep_kernel, one CTA per (sequence, key head, chunk), all in parallel: the
+//     state-independent part. Normalised keys / queries and their Gram matrix (tensor cores),
+//     once for all value heads of the group; per value head, the gates and
 //     then Mo and Keff^T without forming Tm: both solve x (I + A) = y for a row vector y (a row
 //     of Cq, or the column exp(G_C - G_t) khat_t[j] for one key dimension j), which one thread
 //     does by right-looking back substitution in registers. The results go to the workspace in
-//     the exact shared-memory image the scan consumes (one bulk store each).
+//     the exact shared-memory image the scan consumes (the scan copies them in whole).
 //   gdn_prefill_scan_kernel, one CTA per (sequence, value head), chunk after chunk, warp
 //     specialised: warp 8 streams the chunk operands in (bulk copies and a TMA tensor copy of
 //     V) and issues the tensor-core MMAs; warps 0-7 form X and write the outputs. The state
 //     lives in tensor memory (fp32) as the A operand of P | R and the accumulator of the
-//     update. Its per-chunk decay d_C is carried in a scalar sigma (state = sigma * S~) and
+//     update. Two wide MMA chains per chunk ([P | R], N = 128; [O | S update], N = 192): the
+//     tf32 MMA has a large fixed cost per instruction, so fewer, wider ones finish sooner. Its per-chunk decay d_C is carried in a scalar sigma (state = sigma * S~) and
 //     folded into X, so the tensor-memory state is only rescaled when sigma would fall below
 //     2^-32.
 // Precision (kind::tf32 reads operands as truncated tf32): S [Khat; Qhat]^T and the Gram take
@@ -61,8 +63,8 @@ constexpr uint32_t kMaxPolls = 1u << 24;
 //     K-major SWIZZLE_128B image (four 32-column blocks of [128 rows][32]).
 //   Records, one per (sequence, value head, chunk):
 //     B2  [192 rows][64 s] K-major SWIZZLE_128B image (two blocks of [192][32]):
-//         rows 0..127 Keff^T (row j = Keff_s[j] over s), rows 128..191 Mo (row t = Mo[t][s]);
-//         values rounded to the nearest tf32.
+//         rows 0..63 Mo (row t = Mo[t][s]), rows 64..191 Keff^T (row j = Keff_s[j] over s);
+//         values rounded to the nearest tf32. One N = 192 MMA against it gives [O | S update].
 //     vec d[64] | beta[64] | d_C | pad  (144 fp32)
 constexpr int kRecRows = DK + kC;                             // 192
 constexpr uint32_t kKQBytes = 2 * kC * DK * 4;                // 65536
@@ -77,11 +79,18 @@ __host__ __device__ inline size_t n_chunks_of(int T) { return ((size_t)T + kC - 
 // ---------------------------------------------------------------- prep kernel
 
 constexpr int kApad = 68;               // A row stride (floats): 16-byte rows, float4 stores conflict-free
+constexpr float kLog2e = 1.4426950408889634f;
 
+// One CTA per (sequence, key head, chunk): keys / queries, their normalisation and Gram matrix
+// are the same for every value head of the group; gates, decays and the solves are per value
+// head. A and the gate vectors are double-buffered so that warps 0, 1 prepare the next value
+// head while warps 2-7 solve the current one.
 struct __align__(1024) PrepSmem {
-    float KQ[2 * kC * DK];     // [khat; qhat] SW128 image; afterwards the staging of B2
-    float A[kC][kApad];        // strictly lower A
-    float G[kC], Beta[kC], Ec[kC];
+    float KQ[2 * kC * DK];     // [khat; qhat] SW128 image (Gram operands, Keff right-hand sides)
+    float A[2][kC][kApad];     // strictly lower A
+    float G2[2][kC];           // inclusive cumulative log2-decay over the chunk
+    float Beta[2][kC];
+    float Ec[2][kC];           // 2^(G2_{n-1} - G2_t)
     uint64_t mma_done;
     uint32_t tmem;
 };
@@ -104,25 +113,106 @@ __device__ __forceinline__ void solve_unit_lower_row(float2 (&acc)[kC / 2], cons
     }
 }
 
+// Warps 0, 1 (token t = threadIdx.x): the gates of value head h over this chunk into buffer
+// buf (log2 units), and the record's vec (d_t, beta_t, d_C). Named barrier 1 orders the two
+// warps' halves of the prefix sum.
+template <typename InT>
+__device__ __forceinline__ void prep_head_gates(const VerifyArgs& p, PrepSmem& sm, int buf, int b, int h, int t0,
+                                                int n, float* vec) {
+    const int t = threadIdx.x;
+    const int lane = t & 31;
+    float gl = 0.f, be = 0.f;
+    if (t < n) {
+        const size_t gi = ((size_t)b * p.T + t0 + t) * p.Hv + h;
+        gl = -expf(p.A_log[h]) * softplus_f(ld_in<InT>(p.a, gi) + p.dt_bias[h]) * kLog2e;
+        be = 1.f / (1.f + expf(-ld_in<InT>(p.b, gi)));
+    }
+    float Gs = gl;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(kFull, Gs, off);
+        if (lane >= off) Gs += y;
+    }
+    sm.G2[buf][t] = Gs;
+    sm.Beta[buf][t] = be;
+    named_barrier_sync(1, 2 * 32);
+    if (t >= 32) sm.G2[buf][t] = Gs + sm.G2[buf][31];
+    named_barrier_sync(1, 2 * 32);
+    const float GC = sm.G2[buf][n - 1];
+    const float G = sm.G2[buf][t];
+    sm.Ec[buf][t] = t < n ? exp2_approx(GC - G) : 0.f;
+    vec[t] = t < n ? exp2_approx(G) : 0.f;
+    vec[kC + t] = be;
+    if (t == 0) vec[2 * kC] = exp2_approx(GC);
+    named_barrier_sync(1, 2 * 32);
+}
+
+// Warps 0, 1 (row t = threadIdx.x): A[t][s] = beta_t 2^(G2_t - G2_s) Kk[t][s] for s < t, from
+// Gram row t in tensor memory, into A[buf].
+__device__ __forceinline__ void prep_rows_A(PrepSmem& sm, int buf, uint32_t tmem, int n) {
+    const int t = threadIdx.x;
+    float gv[kC];
+#pragma unroll
+    for (int cb = 0; cb < kC; cb += 16)
+        tc::tmem_ld16(tmem + ((uint32_t)(t & ~31) << 16) + cb, *reinterpret_cast<float(*)[16]>(&gv[cb]));
+    const float Gt = sm.G2[buf][t], bt = sm.Beta[buf][t];
+#pragma unroll
+    for (int s4 = 0; s4 < kC; s4 += 4) {
+        float a[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int s = s4 + e;
+            a[e] = (s < t && t < n) ? bt * exp2_approx(Gt - sm.G2[buf][s]) * gv[s] : 0.f;
+        }
+        *reinterpret_cast<float4*>(&sm.A[buf][t][s4]) = make_float4(a[0], a[1], a[2], a[3]);
+    }
+}
+
+// Warps 2-7, the right-hand sides of the solves for the value head in buffer buf. Warps 2, 3
+// (Mo row t = tid - 64): Cq[t][s] = 2^(G2_t - G2_s) Qk[t][s], s <= t, from Gram row 64 + t.
+// Warps 4-7 (key dimension j = tid - 128): Ec_s khat_s[j].
+__device__ __forceinline__ void prep_rhs(const PrepSmem& sm, int buf, uint32_t tmem, int n, float2 (&acc)[kC / 2]) {
+    const int tid = threadIdx.x;
+    if (tid < 128) {
+        float gv[kC];
+#pragma unroll
+        for (int cb = 0; cb < kC; cb += 16)
+            tc::tmem_ld16(tmem + ((uint32_t)(tid & ~31) << 16) + cb, *reinterpret_cast<float(*)[16]>(&gv[cb]));
+        const int t = tid - kC;
+        const float Gt = sm.G2[buf][t];
+#pragma unroll
+        for (int s2 = 0; s2 < kC / 2; ++s2) {
+            const int s = 2 * s2;
+            acc[s2].x = (s <= t && t < n) ? exp2_approx(Gt - sm.G2[buf][s]) * gv[s] : 0.f;
+            acc[s2].y = (s + 1 <= t && t < n) ? exp2_approx(Gt - sm.G2[buf][s + 1]) * gv[s + 1] : 0.f;
+        }
+    } else {
+        const int j = tid - 128;
+#pragma unroll
+        for (int s2 = 0; s2 < kC / 2; ++s2) {
+            const int s = 2 * s2;
+            acc[s2].x = sm.Ec[buf][s] * sm.KQ[tc::sw128_offset(s, j, 2 * kC) / 4];
+            acc[s2].y = sm.Ec[buf][s + 1] * sm.KQ[tc::sw128_offset(s + 1, j, 2 * kC) / 4];
+        }
+    }
+}
+
 template <typename InT>
 __global__ void __launch_bounds__(kPrepThreads, 2)
     gdn_prefill_prep_kernel(const VerifyArgs p, float* __restrict__ ws_kq, unsigned char* __restrict__ ws_rec) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     PrepSmem& sm = *reinterpret_cast<PrepSmem*>(smem_raw);
     const int tid = threadIdx.x;
-    const int lane = tid & 31;
     const int warp = tid >> 5;
     const int c = blockIdx.x;
-    const int h = blockIdx.y;
+    const int g = blockIdx.y;
     const int b = blockIdx.z;
     const int T = p.T;
     const int grp = p.Hv / p.Hk;
-    const int g = h / grp;
     const size_t nch = n_chunks_of(T);
     const int t0 = c * kC;
     const int n = min(kC, T - t0);   // tokens in this chunk
-    const size_t unit = ((size_t)b * p.Hv + h) * nch + c;
-    const bool store_kq = (h % grp) == 0;   // one value head per key head writes the KQ tile
+    auto record = [&](int hh) { return ws_rec + (((size_t)b * p.Hv + (size_t)g * grp + hh) * nch + c) * kRecBytes; };
 
     if ((smem_u32(smem_raw) & 1023u) != 0) {
         if (tid == 0 && p.status_word) atomicOr(p.status_word, kStatusWaitTimeout);
@@ -137,15 +227,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
         tc::tmem_relinquish();
     }
 
-    // 1. Gates of this chunk (warps 0, 1: token t = tid), loads issued first.
-    float gl = 0.f, be = 0.f;
-    if (warp < 2 && tid < n) {
-        const size_t gi = ((size_t)b * T + t0 + tid) * p.Hv + h;
-        gl = -expf(p.A_log[h]) * softplus_f(ld_in<InT>(p.a, gi) + p.dt_bias[h]);
-        be = 1.f / (1.f + expf(-ld_in<InT>(p.b, gi)));
-    }
-    // khat / qhat rows: 16 threads x 8 columns per row, 16 rows per pass, all loads in flight.
+    // 1. Gates of the group's first value head (warps 0, 1), then the khat / qhat rows: 16
+    // threads x 8 columns per row, 16 rows per pass, all loads in flight; written to shared
+    // memory and, as the same SW128 image, to the workspace for the scan.
+    if (warp < 2) prep_head_gates<InT>(p, sm, 0, b, g * grp, t0, n, reinterpret_cast<float*>(record(0) + kB2Bytes));
     {
+        float* kq_dst = ws_kq + (((size_t)b * p.Hk + g) * nch + c) * (kKQBytes / 4);
         const int c16 = tid & 15;
         float x[8][8];
 #pragma unroll
@@ -170,21 +257,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             for (int e = 0; e < 8; ++e) ss = fmaf(x[it][e], x[it][e], ss);
             ss = group_sum<16>(ss);
             const float inv = t < n ? (isq ? p.scale : 1.f) / sqrtf(ss + p.l2_eps) : 0.f;
-            *reinterpret_cast<float4*>(&sm.KQ[tc::sw128_offset(r, 8 * c16, 2 * kC) / 4]) =
-                make_float4(x[it][0] * inv, x[it][1] * inv, x[it][2] * inv, x[it][3] * inv);
-            *reinterpret_cast<float4*>(&sm.KQ[tc::sw128_offset(r, 8 * c16 + 4, 2 * kC) / 4]) =
-                make_float4(x[it][4] * inv, x[it][5] * inv, x[it][6] * inv, x[it][7] * inv);
+            const float4 lo = make_float4(x[it][0] * inv, x[it][1] * inv, x[it][2] * inv, x[it][3] * inv);
+            const float4 hi = make_float4(x[it][4] * inv, x[it][5] * inv, x[it][6] * inv, x[it][7] * inv);
+            const uint32_t o0 = tc::sw128_offset(r, 8 * c16, 2 * kC) / 4;
+            const uint32_t o1 = tc::sw128_offset(r, 8 * c16 + 4, 2 * kC) / 4;
+            *reinterpret_cast<float4*>(&sm.KQ[o0]) = lo;
+            *reinterpret_cast<float4*>(&sm.KQ[o1]) = hi;
+            *reinterpret_cast<float4*>(&kq_dst[o0]) = lo;
+            *reinterpret_cast<float4*>(&kq_dst[o1]) = hi;
         }
-    }
-    if (warp < 2) {
-        float Gs = gl;   // inclusive prefix sum within the warp; warp 1 adds warp 0's total below
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(kFull, Gs, off);
-            if (lane >= off) Gs += y;
-        }
-        sm.G[tid] = Gs;
-        sm.Beta[tid] = be;
     }
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -192,8 +273,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem;
 
-    // 2. Gram on the tensor cores: D (128 x 64) = [Khat; Qhat] Khat^T, one tf32 pass; the KQ
-    // tile goes to the workspace at the same time.
+    // 2. Gram on the tensor cores: D (128 x 64) = [Khat; Qhat] Khat^T, one tf32 pass. It stays
+    // in tensor memory for every value head of the group.
     if (tid == 0) {
         const uint32_t id = tc::idesc_tf32(2 * kC, kC);
         const uint32_t kq = smem_u32(sm.KQ);
@@ -207,94 +288,40 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
             }
         tc::mma_commit(&sm.mma_done);
     }
-    if (tid == 32 && store_kq) {
-        bulk_s2g(ws_kq + (((size_t)b * p.Hk + g) * nch + c) * (kKQBytes / 4), sm.KQ, kKQBytes);
-        bulk_commit();
-    }
-    if (warp == 1) sm.G[tid] += sm.G[31];
-    __syncthreads();
-    if (tid < kC) {
-        const float GC = sm.G[n - 1];
-        sm.Ec[tid] = tid < n ? expf(GC - sm.G[tid]) : 0.f;
-        float* vec = reinterpret_cast<float*>(ws_rec + unit * kRecBytes + kB2Bytes);
-        vec[tid] = tid < n ? expf(sm.G[tid]) : 0.f;
-        vec[kC + tid] = sm.Beta[tid];
-        if (tid == 0) vec[2 * kC] = expf(GC);
-    }
-    __syncthreads();
-
-    // 3. Right-hand sides. Warps 0, 1: Gram rows t -> A row t in shared memory. Warps 2, 3:
-    // Gram rows 64 + t -> Cq row t (registers). Warps 4-7: key dimension j -> exp(G_C - G_s)
-    // khat_s[j] (registers).
-    bool ok = mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls);
+    const bool ok = mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls);
     tc::fence_after_sync();
-    float2 acc[kC / 2];
-    if (warp < 4) {
-        float gv[kC];
-#pragma unroll
-        for (int cb = 0; cb < kC; cb += 16)
-            tc::tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + cb, *reinterpret_cast<float(*)[16]>(&gv[cb]));
-        const int t = (32 * warp + lane) & (kC - 1);
-        const float Gt = sm.G[t];
-        if (warp < 2) {
-            const float bt = sm.Beta[t];
-#pragma unroll
-            for (int s4 = 0; s4 < kC; s4 += 4) {
-                float a[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int s = s4 + e;
-                    a[e] = (s < t && t < n) ? bt * expf(Gt - sm.G[s]) * gv[s] : 0.f;
-                }
-                *reinterpret_cast<float4*>(&sm.A[t][s4]) = make_float4(a[0], a[1], a[2], a[3]);
-            }
-        } else {
-#pragma unroll
-            for (int s2 = 0; s2 < kC / 2; ++s2) {
-                const int s = 2 * s2;
-                acc[s2].x = (s <= t && t < n) ? expf(Gt - sm.G[s]) * gv[s] : 0.f;
-                acc[s2].y = (s + 1 <= t && t < n) ? expf(Gt - sm.G[s + 1]) * gv[s + 1] : 0.f;
-            }
-        }
-    } else {
-        const int j = tid - 128;
-#pragma unroll
-        for (int s2 = 0; s2 < kC / 2; ++s2) {
-            const int s = 2 * s2;
-            acc[s2].x = sm.Ec[s] * sm.KQ[tc::sw128_offset(s, j, 2 * kC) / 4];
-            acc[s2].y = sm.Ec[s + 1] * sm.KQ[tc::sw128_offset(s + 1, j, 2 * kC) / 4];
-        }
-    }
-    if (tid == 32 && store_kq) bulk_wait_read_all();   // the KQ store has read the tile
+    if (warp < 2) prep_rows_A(sm, 0, tmem, n);
     tc::fence_before_sync();
     __syncthreads();
 
-    // 4. Solves: warps 2, 3 give Mo rows, warps 4-7 Keff^T rows; staged (rounded to tf32) over
-    // the KQ tile, which is no longer read, in the record's B2 image.
-    if (ok && warp >= 2) {
-        solve_unit_lower_row(acc, sm.A);
-        const int row = warp < 4 ? DK + (tid - 64) : tid - 128;
+    // 3. Per value head hh: warps 2-7 solve (warps 2, 3 give Mo rows 0..63, warps 4-7 Keff^T
+    // rows 64..191) and write the rows, rounded to tf32, straight into the record's B2 image;
+    // meanwhile warps 0, 1 prepare head hh + 1.
+    for (int hh = 0; hh < grp; ++hh) {
+        const int buf = hh & 1;
+        if (warp >= 2) {
+            float2 acc[kC / 2];
+            prep_rhs(sm, buf, tmem, n, acc);
+            if (ok) {
+                solve_unit_lower_row(acc, sm.A[buf]);
+                const int row = warp < 4 ? tid - 64 : kC + (tid - 128);
+                float* rec = reinterpret_cast<float*>(record(hh));
 #pragma unroll
-        for (int f = 0; f < kC / 4; ++f) {
-            const float4 v = make_float4(tc::tf32_rna(acc[2 * f].x), tc::tf32_rna(acc[2 * f].y),
-                                         tc::tf32_rna(acc[2 * f + 1].x), tc::tf32_rna(acc[2 * f + 1].y));
-            *reinterpret_cast<float4*>(&sm.KQ[tc::sw128_offset(row, 4 * f, kRecRows) / 4]) = v;
+                for (int f = 0; f < kC / 4; ++f) {
+                    const float4 v = make_float4(tc::tf32_rna(acc[2 * f].x), tc::tf32_rna(acc[2 * f].y),
+                                                 tc::tf32_rna(acc[2 * f + 1].x), tc::tf32_rna(acc[2 * f + 1].y));
+                    *reinterpret_cast<float4*>(&rec[tc::sw128_offset(row, 4 * f, kRecRows) / 4]) = v;
+                }
+            }
+        } else if (hh + 1 < grp) {
+            prep_head_gates<InT>(p, sm, buf ^ 1, b, g * grp + hh + 1, t0, n,
+                                 reinterpret_cast<float*>(record(hh + 1) + kB2Bytes));
+            prep_rows_A(sm, buf ^ 1, tmem, n);
         }
+        tc::fence_before_sync();
+        __syncthreads();
     }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        if (ok) {
-            bulk_s2g(ws_rec + unit * kRecBytes, sm.KQ, kB2Bytes);
-            bulk_commit();
-            bulk_wait_all();
-        } else if (p.status_word) {
-            atomicOr(p.status_word, kStatusWaitTimeout);
-        }
-    }
-    if (tid == 32 && store_kq) bulk_wait_all();
-    tc::fence_before_sync();
-    __syncthreads();
+    if (!ok && tid == 0 && p.status_word) atomicOr(p.status_word, kStatusWaitTimeout);
     if (warp == 0) tc::tmem_dealloc(tmem, 64);
 }
 
@@ -315,16 +342,16 @@ __host__ __device__ constexpr uint32_t scan_smem_bytes() { return kOffV0 + 2 * v
 
 struct ScanBars {
     uint64_t kq_full, rec_full[2], v_full[2];
-    uint64_t mma_p, mma_r, mma_s, mma_o, drain;
+    uint64_t mma_pr, mma_so, drain;
     uint64_t x_ready, o_free;           // 256 arrivals each
     uint32_t tmem;
     int abort;
 };
 static_assert(kOffBar + sizeof(ScanBars) <= kOffRec1, "barriers overflow the record slack");
 
-// TMEM columns: S~ 0..127, P 128..191, R (two buffers) 192..319, O 320..383, X_hi 384..447,
-// X_lo 448..511.
-constexpr uint32_t kColS = 0, kColP = 128, kColR = 192, kColO = 320, kColXh = 384, kColXl = 448;
+// TMEM columns: [O | S~] 0..191 (one N = 192 accumulator: O 0..63, S~ 64..191), [P | R]
+// 256..383, X_hi 384..447, X_lo 448..511 (each accumulator starts at a multiple of its width).
+constexpr uint32_t kColO = 0, kColS = 64, kColPR = 256, kColXh = 384, kColXl = 448;
 constexpr float kRenormBelow = 2.3283064365386963e-10f;   // 2^-32
 
 // Bounded wait that also gives up once another thread of the CTA has given up.
@@ -352,27 +379,10 @@ __device__ __forceinline__ void mma_ts_k(uint32_t d, uint32_t a0, uint64_t b0, u
     }
 }
 
-// Outputs of chunk c for state row `row`, tokens 32 half .. +31 (those below n):
-// o_t = rd_t R~_t + divO O'_t, with R~ in tensor-memory buffer c % 2 and O' in the O columns.
-template <typename OutT>
-__device__ __forceinline__ void scan_outputs(const VerifyArgs& p, uint32_t lb, int b, int h, int half, int row, int c,
-                                             int n, const float (&rd)[32], float divO) {
-    OutT* op = reinterpret_cast<OutT*>(p.o);
-    const size_t base = ((size_t)b * p.T + (size_t)c * kC + 32 * half) * p.Hv + h;
-    const uint32_t rcol = kColR + (uint32_t)(c & 1) * kC + 32 * half;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        float rv[16], ov[16];
-        tc::tmem_ld16(lb + rcol + 16 * q, rv);
-        tc::tmem_ld16(lb + kColO + 32 * half + 16 * q, ov);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int u = 16 * q + e;
-            if (32 * half + u < n)
-                st_out<OutT>(op, (base + (size_t)u * p.Hv) * DV + row, fmaf(rd[u], rv[e], divO * ov[e]));
-        }
-    }
-}
+// The decay bookkeeping shared by producer and consumers (identical fp32 arithmetic on both
+// sides): sigma_next = sigma d_C; below 2^-32 (or not a number) the decay is folded into S~
+// instead and sigma restarts at 1.
+__device__ __forceinline__ bool decay_renorm(float snext) { return !(snext >= kRenormBelow); }
 
 template <typename InT, typename OutT>
 __global__ void __launch_bounds__(kScanThreads, 1)
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     constexpr uint32_t kVBytes = v_tile_bytes<InT>();
     ScanBars& bar = *reinterpret_cast<ScanBars*>(smem_raw + kOffBar);
     float* KQ = reinterpret_cast<float*>(smem_raw + kOffKQ);
-    // Record buffer i at smem_raw + kOffRec0 + i * kRecStride, V buffer i at kOffV0 + i * kVBytes.
+    // Record buffer i at kOffRec0 + i * kRecStride, V buffer i at kOffV0 + i * kVBytes.
     auto REC = [&](int i) { return smem_raw + kOffRec0 + (uint32_t)i * kRecStride; };
     auto VT = [&](int i) { return smem_raw + kOffV0 + (uint32_t)i * kVBytes; };
     volatile int* abort = &bar.abort;
@@ -410,10 +420,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         mbar_init(&bar.rec_full[1], 1);
         mbar_init(&bar.v_full[0], 1);
         mbar_init(&bar.v_full[1], 1);
-        mbar_init(&bar.mma_p, 1);
-        mbar_init(&bar.mma_r, 1);
-        mbar_init(&bar.mma_s, 1);
-        mbar_init(&bar.mma_o, 1);
+        mbar_init(&bar.mma_pr, 1);
+        mbar_init(&bar.mma_so, 1);
         mbar_init(&bar.drain, 1);
         mbar_init(&bar.x_ready, 256);
         mbar_init(&bar.o_free, 256);
@@ -466,7 +474,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const int row = 32 * q4 + lane;
     const uint32_t lb = tmem + ((uint32_t)(32 * q4) << 16);
 
-    // Initial state (zero when state_in is NULL) into tensor memory, columns 64 half .. +63.
+    // Initial state (zero when state_in is NULL) into tensor memory, columns 64 half .. +63 of
+    // S~, and zeros in this thread's O columns.
     if (warp < 8) {
         const float* src = p.state_in ? p.state_in + (head * DV + row) * DK + 64 * half : nullptr;
 #pragma unroll
@@ -483,6 +492,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             }
             tc::tmem_st32(lb + kColS + 64 * half + 32 * cb, v);
         }
+        float z[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) z[e] = 0.f;
+        tc::tmem_st32(lb + kColO + 32 * half, z);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -491,97 +504,95 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     bool ok = true;
     if (producer) {
         // ---------------- producer / MMA issuer
-        const uint32_t idPR = tc::idesc_tf32(DV, kC), idS = tc::idesc_tf32(DV, DK), idO = tc::idesc_tf32(DV, kC);
+        const uint32_t idPR = tc::idesc_tf32(DV, 2 * kC), idSO = tc::idesc_tf32(DV, kRecRows);
         const uint64_t dKQ = tc::desc_kmajor_sw128(smem_u32(KQ));
-        auto issue_o = [&](int c) {   // O_c = X'_c Mo_c^T, two passes
-            const uint64_t dMo = tc::desc_kmajor_sw128(smem_u32(REC(c & 1)) + DK * 128);
-            mma_ts_k(tmem + kColO, tmem + kColXh, dMo, kRBlock, 2, idO, false);
-            mma_ts_k(tmem + kColO, tmem + kColXl, dMo, kRBlock, 2, idO, true);
-            tc::mma_commit(&bar.mma_o);
-        };
-        for (int c = 0; c < nch && ok; ++c) {
+        float sigma = 1.f;   // mirrors the consumers' decay scalar
+        for (int c = 0; c < nch; ++c) {
             if (!wait_or_abort(&bar.kq_full, c & 1, abort)) { ok = false; break; }
+            // S~ is final once the previous update is done.
+            if (c >= 1 && !wait_or_abort(&bar.mma_so, (c - 1) & 1, abort)) { ok = false; break; }
             tc::fence_after_sync();
-            // P_c = S~ Khat^T, then R_c = S~ Qhat^T (A = S~ in tensor memory, one pass).
-            mma_ts_k(tmem + kColP, tmem + kColS, dKQ, kKBlock, 4, idPR, false);
-            tc::mma_commit(&bar.mma_p);
-            // R_c and O_{c-1} overwrite what the outputs of chunk c-2 read, and the record
-            // buffer refilled below held the vec the consumers copied in chunk c-1.
-            if (c >= 1 && !wait_or_abort(&bar.o_free, (c - 1) & 1, abort)) { ok = false; break; }
-            mma_ts_k(tmem + kColR + (uint32_t)(c & 1) * kC, tmem + kColS, dKQ + ((kC * 128) >> 4), kKBlock, 4, idPR,
-                     false);
-            tc::mma_commit(&bar.mma_r);
-            if (c >= 1) issue_o(c - 1);
-            // The KQ tile is free once R_c is done.
-            if (!wait_or_abort(&bar.mma_r, c & 1, abort)) { ok = false; break; }
-            if (c + 1 < nch) load_kq(c + 1);
-            // Record buffer (c + 1) & 1 is free once O_{c-1} is done.
+            // [P | R]_c = S~ [Khat; Qhat]^T (A = S~ in tensor memory, one pass, N = 128).
+            mma_ts_k(tmem + kColPR, tmem + kColS, dKQ, kKBlock, 4, idPR, false);
+            tc::mma_commit(&bar.mma_pr);
+            // Record buffer (c + 1) & 1 held chunk c - 1: its operands were read by the
+            // previous update, its vec by the consumers' outputs of chunk c - 1.
             if (c >= 1) {
-                if (!wait_or_abort(&bar.mma_o, (c - 1) & 1, abort)) { ok = false; break; }
+                if (!wait_or_abort(&bar.o_free, (c - 1) & 1, abort)) { ok = false; break; }
                 if (c + 1 < nch) load_rec(c + 1);
             }
-            // S~ += X'_c Keff_c, two passes, once X'_c is in tensor memory.
+            // The KQ tile is free once [P | R]_c is done.
+            if (!wait_or_abort(&bar.mma_pr, c & 1, abort)) { ok = false; break; }
+            if (c + 1 < nch) load_kq(c + 1);
+            // [O | S~] (+)= X'_c [Mo; Keff^T]^T, two passes (X_hi, X_lo), N = 192, once X'_c is
+            // in tensor memory. A state decayed to exactly zero is overwritten, not rescaled
+            // (the O columns were zeroed by the consumers, so they start fresh either way).
             if (!wait_or_abort(&bar.x_ready, c & 1, abort)) { ok = false; break; }
             if (!wait_or_abort(&bar.rec_full[c & 1], (c >> 1) & 1, abort)) { ok = false; break; }
             tc::fence_after_sync();
-            {
-                const uint64_t dKe = tc::desc_kmajor_sw128(smem_u32(REC(c & 1)));
-                mma_ts_k(tmem + kColS, tmem + kColXh, dKe, kRBlock, 2, idS, true);
-                mma_ts_k(tmem + kColS, tmem + kColXl, dKe, kRBlock, 2, idS, true);
-                tc::mma_commit(&bar.mma_s);
-            }
+            const float dC = reinterpret_cast<const float*>(REC(c & 1) + kB2Bytes)[2 * kC];
+            const float snext = sigma * dC;
+            sigma = decay_renorm(snext) ? 1.f : snext;
+            const uint64_t dB2 = tc::desc_kmajor_sw128(smem_u32(REC(c & 1)));
+            mma_ts_k(tmem + kColO, tmem + kColXh, dB2, kRBlock, 2, idSO, snext != 0.f);
+            mma_ts_k(tmem + kColO, tmem + kColXl, dB2, kRBlock, 2, idSO, true);
+            tc::mma_commit(&bar.mma_so);
             if (c + 2 < nch) load_v(c + 2);   // V_c was read before x_ready
-            if (!wait_or_abort(&bar.mma_s, c & 1, abort)) { ok = false; break; }
-        }
-        if (ok) {
-            if (wait_or_abort(&bar.o_free, (nch - 1) & 1, abort)) issue_o(nch - 1);
-            else ok = false;
         }
     } else if (warp < 8) {
         // ---------------- consumers
         float sigma = 1.f;      // state = sigma * S~
-        float rd[32];           // sigma_c d_t for the previous chunk's outputs
-        float divO = 1.f;       // O = divO * (X' Mo^T) for the previous chunk
-        int n_prev = 0;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) rd[e] = 0.f;
+        OutT* op = reinterpret_cast<OutT*>(p.o);
         for (int c = 0; c < nch; ++c) {
-            const int t0 = c * kC;
-            const int n = min(kC, T - t0);
+            const int n = min(kC, T - c * kC);
             const int s = c & 1;
             const float* vec = reinterpret_cast<const float*>(REC(s) + kB2Bytes);
             if (!wait_or_abort(&bar.rec_full[s], (c >> 1) & 1, abort)) { ok = false; break; }
             const float dC = vec[2 * kC];
             const float snext = sigma * dC;
-            const bool renorm = !(snext >= kRenormBelow);
+            const bool renorm = decay_renorm(snext);
             const float inv = renorm ? 1.f : 1.f / snext;
-            if (!wait_or_abort(&bar.mma_p, c & 1, abort)) { ok = false; break; }
+            if (!wait_or_abort(&bar.mma_pr, c & 1, abort)) { ok = false; break; }
             tc::fence_after_sync();
             if (!wait_or_abort(&bar.v_full[s], (c >> 1) & 1, abort)) { ok = false; break; }
+            // R~_c (kept for this chunk's outputs) and P~_c, both loaded before one wait.
+            float rv[32], pv[32];
+            tc::tmem_ld32x2(lb + kColPR + kC + 32 * half, lb + kColPR + 32 * half, rv, pv);
+            // X'_s = beta_s inv (v_s - sigma d_s P~_s) = a_s v_s - a_s sigma d_s P~_s with
+            // a_s = beta_s inv, split into its tf32 high part and the remainder, two tokens per
+            // packed fp32 instruction.
             const InT* vt = reinterpret_cast<const InT*>(VT(s)) + row;
-            // X'_s = beta_s inv (v_s - sigma d_s P~_s), split into tf32 high part and remainder.
+            const float2 inv2 = make_float2(inv, inv), sig2 = make_float2(sigma, sigma);
             float xh[32], xl[32];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                float pv[16];
-                tc::tmem_ld16(lb + kColP + 32 * half + 16 * q, pv);
+            for (int f = 0; f < 8; ++f) {
+                const int t = 32 * half + 4 * f;
+                const float4 be = *reinterpret_cast<const float4*>(&vec[kC + t]);
+                const float4 dd = *reinterpret_cast<const float4*>(&vec[t]);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int t = 32 * half + 16 * q + e;
-                    const float x = vec[kC + t] * inv * fmaf(-vec[t] * sigma, pv[e], to_f(vt[t * DV]));
-                    xh[16 * q + e] = tc::tf32_hi(x);
-                    xl[16 * q + e] = x - xh[16 * q + e];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int e = 4 * f + 2 * hh;
+                    const float2 a2 = __fmul2_rn(hh ? make_float2(be.z, be.w) : make_float2(be.x, be.y), inv2);
+                    const float2 bq =
+                        __fmul2_rn(__fmul2_rn(a2, sig2), hh ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y));
+                    const float2 v2 = make_float2(to_f(vt[(t + 2 * hh) * DV]), to_f(vt[(t + 2 * hh + 1) * DV]));
+                    const float2 x2 =
+                        __ffma2_rn(make_float2(-bq.x, -bq.y), make_float2(pv[e], pv[e + 1]), __fmul2_rn(a2, v2));
+                    xh[e] = tc::tf32_hi(x2.x);
+                    xh[e + 1] = tc::tf32_hi(x2.y);
+                    const float2 l2 = __fadd2_rn(x2, make_float2(-xh[e], -xh[e + 1]));
+                    xl[e] = l2.x;
+                    xl[e + 1] = l2.y;
                 }
             }
-            // X_{c-1} must have been read by O_{c-1} before it is overwritten.
-            if (c >= 1) {
-                if (!wait_or_abort(&bar.mma_o, (c - 1) & 1, abort)) { ok = false; break; }
-                tc::fence_after_sync();
-            }
-            if (renorm) {
-                // Fold sigma d_C into S~ itself (R_c must have read S~ first); X' = X.
-                if (!wait_or_abort(&bar.mma_r, c & 1, abort)) { ok = false; break; }
-                tc::fence_after_sync();
+            tc::tmem_st16_nowait(lb + kColXh + 32 * half, &xh[0]);
+            tc::tmem_st16_nowait(lb + kColXh + 32 * half + 16, &xh[16]);
+            tc::tmem_st16_nowait(lb + kColXl + 32 * half, &xl[0]);
+            tc::tmem_st16_nowait(lb + kColXl + 32 * half + 16, &xl[16]);
+            tc::tmem_st_wait();
+            if (renorm && snext != 0.f) {
+                // Fold sigma d_C into S~ itself ([P | R]_c has read it); X' = X. A decay of
+                // exactly zero is left to the producer, which overwrites S~.
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
                     float sv[32];
@@ -593,23 +604,47 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     tc::tmem_st32(col, sv);
                 }
             }
-            tc::tmem_st32(lb + kColXh + 32 * half, xh);
-            tc::tmem_st32(lb + kColXl + 32 * half, xl);
             tc::fence_before_sync();
             mbar_arrive(&bar.x_ready);
-            if (c >= 1) scan_outputs<OutT>(p, lb, b, h, half, row, c - 1, n_prev, rd, divO);
+            // Outputs of this chunk once [O | S~]_c is done: o_t = sigma_c d_t R~_t + divO O'_t,
+            // tokens 32 half .. +31; the O columns are zeroed again for the next chunk.
+            if (!wait_or_abort(&bar.mma_so, c & 1, abort)) { ok = false; break; }
+            tc::fence_after_sync();
+            float ov[32];
+            tc::tmem_ld16(lb + kColO + 32 * half, *reinterpret_cast<float(*)[16]>(&ov[0]));
+            tc::tmem_ld16(lb + kColO + 32 * half + 16, *reinterpret_cast<float(*)[16]>(&ov[16]));
+            {
+                float z[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rd[e] = sigma * vec[32 * half + e];
-            divO = renorm ? 1.f : snext;
+                for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                tc::tmem_st32(lb + kColO + 32 * half, z);
+            }
+            const float divO = renorm ? 1.f : snext;
+            const float2 div2 = make_float2(divO, divO), sig2o = make_float2(sigma, sigma);
+            const size_t tstride = (size_t)p.Hv * DV;   // elements between consecutive tokens
+            OutT* orow = op + (((size_t)b * T + (size_t)c * kC + 32 * half) * p.Hv + h) * DV + row;
+            const int nt = n - 32 * half;                // tokens of this half inside the prompt
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+                const float4 dd = *reinterpret_cast<const float4*>(&vec[32 * half + 4 * f]);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int e = 4 * f + 2 * hh;
+                    const float2 rd = __fmul2_rn(sig2o, hh ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y));
+                    const float2 y = __ffma2_rn(rd, make_float2(rv[e], rv[e + 1]),
+                                                __fmul2_rn(div2, make_float2(ov[e], ov[e + 1])));
+                    if (e < nt) st_out<OutT>(orow, 0, y.x);
+                    orow += tstride;
+                    if (e + 1 < nt) st_out<OutT>(orow, 0, y.y);
+                    orow += tstride;
+                }
+            }
             sigma = renorm ? 1.f : snext;
-            n_prev = n;
             tc::fence_before_sync();
             mbar_arrive(&bar.o_free);
         }
-        if (ok && wait_or_abort(&bar.mma_o, (nch - 1) & 1, abort)) {
-            tc::fence_after_sync();
-            scan_outputs<OutT>(p, lb, b, h, half, row, nch - 1, n_prev, rd, divO);
-            // Final state = sigma S~.
+        if (ok) {
+            // Final state = sigma S~ (the last update was waited for above).
             float* dst = p.state_out + (head * DV + row) * DK + 64 * half;
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
@@ -621,8 +656,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                     reinterpret_cast<float4*>(dst + 32 * cb)[q] =
                         make_float4(sigma * v[4 * q], sigma * v[4 * q + 1], sigma * v[4 * q + 2], sigma * v[4 * q + 3]);
             }
-        } else {
-            ok = false;
         }
     }
     if (!ok) *abort = 1;
@@ -660,7 +693,7 @@ cudaError_t launch_tc_prefill(const VerifyArgs& a, void* workspace, cudaStream_t
     CUtensorMap v_map;
     e = tc::encode_tmap_tokens(&v_map, a.v, sizeof(InT) == 2, DV, a.Hv, a.T, a.B, kC);
     if (e != cudaSuccess) return e;
-    dim3 pgrid((unsigned)nch, a.Hv, a.B);
+    dim3 pgrid((unsigned)nch, a.Hk, a.B);
     gdn_prefill_prep_kernel<InT><<<pgrid, kPrepThreads, sizeof(PrepSmem), stream>>>(a, ws_kq, ws_rec);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

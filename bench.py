@@ -34,29 +34,36 @@ from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload  # noq
 METRIC = "GDN verify/decode HBM GB/s (frac of B200 peak), token·heads/s; prefill tok/s"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-# Sources of the dominant kernels; a committed ncu traffic figure is only reported while
-# these are unchanged.
-KERNEL_SOURCES = ["gated_deltanet_mixer_verify_b200/csrc/gdn_verify.cu",
-                  "gated_deltanet_mixer_verify_b200/csrc/gdn_verify_tc.cu",
-                  "gated_deltanet_mixer_verify_b200/csrc/gdn_verify_head.cu",
-                  "gated_deltanet_mixer_verify_b200/csrc/gdn_tc.cuh",
-                  "gated_deltanet_mixer_verify_b200/csrc/gdn_device.cuh",
-                  "gated_deltanet_mixer_verify_b200/csrc/gdn_internal.cuh"]
+NOMINAL_TF32_OVER_BF16 = 1.1 / 2.25     # dense tensor-core peaks, tf32 vs bf16
+# Sources of each workload's dominant kernel (with the headers it includes); a committed ncu
+# traffic figure is only reported while these are unchanged.
+_CSRC = "gated_deltanet_mixer_verify_b200/csrc/"
+_HEADERS = [_CSRC + f for f in ("gdn_tc.cuh", "gdn_device.cuh", "gdn_internal.cuh")]
+KERNEL_SOURCES = {
+    "batched_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
+    "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
+    "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
+    "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
+}
 
 
 # ----------------------------------------------------------------------------- helpers
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, source) from MEASURED_PEAKS.json, else the fallbacks."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(workload_name: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[workload_name]:
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
@@ -68,7 +75,7 @@ def ncu_traffic(workload_name: str):
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(workload_name)
-    if not d or d.get("kernel_source_sha") != kernel_source_hash():
+    if not d or d.get("kernel_source_sha") != kernel_source_hash(workload_name):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -242,6 +249,7 @@ class SingleSeq:
 
 class Prefill:
     tokens = 0   # prompt length override (0: the workload's)
+    dtype = "tf32"   # tensor-core products in tf32 (one or two passes), solves in fp32
 
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
@@ -249,24 +257,39 @@ class Prefill:
         self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
         if Prefill.tokens:
             self.w = workload(name, seed=self.w.seed, T=Prefill.tokens)
-        x = make_inputs(self.w)
-        self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        self.host = make_inputs(self.w)
+        self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.host.items()}
         w = self.w
         self.o = torch.empty(self.x["v"].shape, dtype=torch.float32, device=dev)
         self.state = torch.empty((w.B, w.H_v, w.d_v, w.d_k), dtype=torch.float32, device=dev)
         nb = gdn.prefill_workspace_bytes(w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v, w.chunk)
         self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
-        self.launches_per_step = 1
-        el = 2
-        self.bytes = (2 * w.B * w.T * w.H_k * w.d_k * el + w.B * w.T * w.H_v * w.d_v * el
-                      + 2 * w.B * w.T * w.H_v * el + w.B * w.T * w.H_v * w.d_v * 4
-                      + w.B * w.H_v * w.d_v * w.d_k * 4)
+        self.launches_per_step = 2          # the prepare kernel and the scan kernel
         self.units = w.B * w.T
+        C, dk, dv = w.chunk, w.d_k, w.d_v
+        n_units = w.B * w.H_v * ((w.T + C - 1) // C)
+        # Algorithmic work per (sequence, value head, chunk). Scan (tensor cores, counted once
+        # however many tf32 passes carry it): [P | R] = S [Khat; Qhat]^T, the state update
+        # X Keff and the outputs X Mo^T. Prepare (CUDA cores): the 192 triangular row solves
+        # giving Mo and Keff^T, 63 * 64 / 2 fused multiply-adds each.
+        self.phase_names = ["prepare", "scan"]
+        self.phase_work = [n_units * 192 * (63 * 64 // 2) * 2,
+                           n_units * (2 * dv * dk * 2 * C + 2 * dv * C * dk + 2 * dv * C * C)]
+        self.phase_kernel = ["gdn_prefill_prep_kernel", "gdn_prefill_scan_kernel"]
 
-    def step(self):
-        x = self.x
-        self.gdn.chunk_prefill(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
-                               None, self.state, self.o, self.w.chunk, self.ws)
+    def phases(self, x=None):
+        x = self.x if x is None else x
+        g, w = self.gdn, self.w
+        return [lambda: g.chunk_prefill_prepare(x["q"], x["k"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                                                self.ws, chunk=w.chunk),
+                lambda: g.chunk_prefill_scan(x["v"], self.ws, w.H_k, None, self.state, self.o, chunk=w.chunk)]
+
+    def step(self, x=None):
+        for ph in self.phases(x):
+            ph()
+
+    def per_step_inputs(self):
+        return ["q", "k", "v", "a", "b"]
 
     def config(self):
         c = workload_config(self.w.name)
@@ -409,9 +432,11 @@ def main():
         wl.step()
     torch.cuda.synchronize(dev)
 
-    # timed region: K steps, device events on the launching stream, per-launch events too
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # timed region: K steps, device events on the launching stream, one more event after each
+    # phase of a step where the workload runs in phases (prefill: prepare, scan)
+    phases = wl.phases() if hasattr(wl, "phases") else None
+    nph = len(phases) if phases else 1
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -419,18 +444,24 @@ def main():
         start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            wl.step()
-            ev[i][1].record(stream)
+            if phases:
+                for j, ph in enumerate(phases):
+                    ph()
+                    ev[i][j + 1].record(stream)
+            else:
+                wl.step()
+                ev[i][1].record(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(end))
-    step_ms = [a.elapsed_time(b) for a, b in ev]
+    step_ms = [e[0].elapsed_time(e[nph]) for e in ev]
+    phase_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) for j in range(nph)]
     ms_per_step = elapsed_ms / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> mixer -> host output
     e2e = None
-    if isinstance(wl, Verify):
+    if isinstance(wl, (Verify, Prefill)):
         names = wl.per_step_inputs()
         host = {k: wl.host[k].pin_memory() for k in names}
         dev_in = dict(wl.x)
@@ -450,36 +481,57 @@ def main():
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = max_over_ranks(e_start.elapsed_time(e_end))
-        e2e = {"value": weak_scaling_throughput(wl.bytes, world, e_ms / args.steps / 1e3) / 1e9,
-               "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        e_s = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps / 1e3
+        if isinstance(wl, Prefill):
+            e2e = {"value": weak_scaling_throughput(wl.units, world, e_s), "unit": "tok/s"}
+        else:
+            e2e = {"value": weak_scaling_throughput(wl.bytes, world, e_s) / 1e9, "unit": "GB/s"}
+        e2e.update({"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h})
 
     if rank == 0:
-        peak, peak_kind = measured_peaks()
-        if args.workload == "prefill":
+        hbm_peak, bf16_peak, peak_kind = measured_peaks()
+        src = "MEASURED_PEAKS.json" if peak_kind == "measured" else "fallback"
+        if isinstance(wl, Prefill):
             value = weak_scaling_throughput(wl.units, world, ms_per_step / 1e3)
             unit = "tok/s"
+            # dominant phase: the scan is tensor-core work against the tf32 peak (the measured
+            # bf16 peak times the nominal tf32 / bf16 ratio); the prepare phase is fp32 FMA work
+            # against 148 SMs x 128 lanes x 2 flop x the maximum SM clock
+            k = max(range(nph), key=lambda j: phase_ms[j])
+            achieved = wl.phase_work[k] / (phase_ms[k] / 1e3) / 1e12
+            if wl.phase_names[k] == "scan":
+                bound, peak = "tensor", bf16_peak * NOMINAL_TF32_OVER_BF16
+                peak_source = "%s bf16_tflops x nominal tf32/bf16 (1.1/2.25), %s" % (src, peak_kind)
+            else:
+                bound, peak = "alu", 148 * 128 * 2 * 1965e6 / 1e12
+                peak_source = "148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz"
+            roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                        "frac": achieved / peak, "peak_source": peak_source,
+                        "traffic": ncu_traffic(args.workload), "kernel": wl.phase_kernel[k],
+                        "algorithmic_flops_per_launch": wl.phase_work[k],
+                        "phase_ms": dict(zip(wl.phase_names, phase_ms))}
+            dtype = Prefill.dtype
         else:
             value = weak_scaling_throughput(wl.bytes, world, ms_per_step / 1e3) / 1e9
             unit = "GB/s"
-        kernel_ms = statistics.mean(step_ms) / wl.launches_per_step
-        per_launch_bytes = wl.bytes / wl.launches_per_step
-        achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
+            kernel_ms = statistics.mean(step_ms) / wl.launches_per_step
+            per_launch_bytes = wl.bytes / wl.launches_per_step
+            achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
+            roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                        "frac": achieved / hbm_peak, "peak_source": "%s hbm_gbs (%s)" % (src, peak_kind),
+                        "traffic": ncu_traffic(args.workload),
+                        "algorithmic_bytes_per_launch": per_launch_bytes}
+            dtype = "f32"
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
             "data": "synthetic", "config": dict(wl.config(), parallelism="dp%d" % world),
             "token_heads_per_s": wl.units * world / (ms_per_step / 1e3)
-            if args.workload != "prefill" else None,
+            if not isinstance(wl, Prefill) else None,
             "frac_of_spec_8TBps": (wl.bytes * world / (ms_per_step / 1e3) / 1e9 / world) / SPEC_HBM_GBS
-            if args.workload != "prefill" else None,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
-                         if peak_kind == "measured" else "fallback 6650 GB/s",
-                         "traffic": ncu_traffic(args.workload),
-                         "algorithmic_bytes_per_launch": per_launch_bytes},
+            if not isinstance(wl, Prefill) else None,
+            "roofline": roofline,
             "clocks": clk.summary(),
             "gpu_launches": args.steps * wl.launches_per_step,
             "e2e": e2e,

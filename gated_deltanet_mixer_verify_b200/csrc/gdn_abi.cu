@@ -207,18 +207,39 @@ size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk) 
     return gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k, shape->d_v, chunk);
 }
 
+// Shape, chunk and workspace checks shared by the workspace-taking prefill entry points.
+// Returns GDN_OK with *empty set when the batch is empty (nothing to launch).
+static gdn_status prefill_checks(const gdn_shape* shape, int32_t chunk, const void* workspace, size_t workspace_bytes,
+                                 const char* who, bool* empty) {
+    *empty = false;
+    if (!shape) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
+    gdn_status st = check_shape(shape, 1 << 30, who);
+    if (st != GDN_OK) return st;
+    if (gdn::check_prefill_shape(shape, chunk) != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: only chunk 64 with d_k = d_v = 128 is built", who);
+    if (shape->B == 0) {
+        *empty = true;
+        return ok();
+    }
+    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k,
+                                                     shape->d_v, chunk);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", who, need,
+                        workspace_bytes);
+        if (!aligned16(workspace)) return fail(GDN_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", who);
+    }
+    return GDN_OK;
+}
+
 gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,
                              const void* v, const void* a, const void* b, const float* A_log,
                              const float* dt_bias, const float* state_in, float* state_out, void* o,
                              void* workspace, size_t workspace_bytes, void* stream) {
     const char* who = "gdn_chunk_prefill";
-    if (!shape) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
-    gdn_status st = check_shape(shape, 1 << 30, who);
-    if (st != GDN_OK) return st;
-    int pc = gdn::check_prefill_shape(shape, chunk);
-    if (pc != 0)
-        return fail(GDN_ERR_UNSUPPORTED, "%s: only chunk 64 with d_k = d_v = 128 is built", who);
-    if (shape->B == 0) return ok();
+    bool empty = false;
+    gdn_status st = prefill_checks(shape, chunk, workspace, workspace_bytes, who, &empty);
+    if (st != GDN_OK || empty) return st;
     REQUIRE_PTR(q, who);
     REQUIRE_PTR(k, who);
     REQUIRE_PTR(v, who);
@@ -233,14 +254,6 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* 
         if (!overlap_ok(state_in, state_out, state_bytes(shape)))
             return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
     }
-    const size_t need = gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k,
-                                                     shape->d_v, chunk);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need)
-            return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", who, need,
-                        workspace_bytes);
-        if (!aligned16(workspace)) return fail(GDN_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", who);
-    }
     gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
     x.state_in = state_in;
     x.state_out = state_out;
@@ -249,6 +262,46 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk, const void* 
     return launched(gdn::launch_prefill(x, chunk, workspace, workspace_bytes,
                                         static_cast<cudaStream_t>(stream)),
                     who);
+}
+
+gdn_status gdn_chunk_prefill_prepare(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,
+                                     const void* a, const void* b, const float* A_log, const float* dt_bias,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    const char* who = "gdn_chunk_prefill_prepare";
+    bool empty = false;
+    gdn_status st = prefill_checks(shape, chunk, workspace, workspace_bytes, who, &empty);
+    if (st != GDN_OK || empty) return st;
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    gdn::VerifyArgs x = make_args(shape, q, k, nullptr, a, b, A_log, dt_bias);
+    return launched(gdn::launch_prefill_prepare(x, workspace, static_cast<cudaStream_t>(stream)), who);
+}
+
+gdn_status gdn_chunk_prefill_scan(const gdn_shape* shape, int32_t chunk, const void* v, const float* state_in,
+                                  float* state_out, void* o, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    const char* who = "gdn_chunk_prefill_scan";
+    bool empty = false;
+    gdn_status st = prefill_checks(shape, chunk, workspace, workspace_bytes, who, &empty);
+    if (st != GDN_OK || empty) return st;
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(state_out, who);
+    REQUIRE_PTR(o, who);
+    if (state_in) {
+        REQUIRE_PTR(state_in, who);
+        if (!overlap_ok(state_in, state_out, state_bytes(shape)))
+            return fail(GDN_ERR_INVALID_ARG, "%s: state_out partially overlaps state_in", who);
+    }
+    gdn::VerifyArgs x = make_args(shape, nullptr, nullptr, v, nullptr, nullptr, nullptr, nullptr);
+    x.state_in = state_in;
+    x.state_out = state_out;
+    x.o = o;
+    x.always_commit = 1;
+    return launched(gdn::launch_prefill_scan(x, workspace, static_cast<cudaStream_t>(stream)), who);
 }
 
 gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk, const void* q, const void* k,

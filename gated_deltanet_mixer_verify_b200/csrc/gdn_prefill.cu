@@ -678,28 +678,35 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-template <typename InT, typename OutT>
-cudaError_t launch_tc_prefill(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
-    const size_t nch = n_chunks_of(a.T);
-    float* ws_kq = static_cast<float*>(workspace);
-    unsigned char* ws_rec = static_cast<unsigned char*>(workspace) + (size_t)a.B * a.Hk * nch * kKQBytes;
+// Workspace pointers: KQ tiles first, then the records.
+inline float* ws_kq_of(const VerifyArgs&, void* ws) { return static_cast<float*>(ws); }
+inline unsigned char* ws_rec_of(const VerifyArgs& a, void* ws) {
+    return static_cast<unsigned char*>(ws) + (size_t)a.B * a.Hk * n_chunks_of(a.T) * kKQBytes;
+}
+
+template <typename InT>
+cudaError_t launch_prep(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
     // Per call: the attribute belongs to the function on the current device.
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_prep_kernel<InT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(PrepSmem));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(gdn_prefill_scan_kernel<InT, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)scan_smem_bytes<InT>());
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)n_chunks_of(a.T), a.Hk, a.B);
+    gdn_prefill_prep_kernel<InT><<<grid, kPrepThreads, sizeof(PrepSmem), stream>>>(a, ws_kq_of(a, workspace),
+                                                                                    ws_rec_of(a, workspace));
+    return cudaGetLastError();
+}
+
+template <typename InT, typename OutT>
+cudaError_t launch_scan(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_scan_kernel<InT, OutT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem_bytes<InT>());
     if (e != cudaSuccess) return e;
     CUtensorMap v_map;
     e = tc::encode_tmap_tokens(&v_map, a.v, sizeof(InT) == 2, DV, a.Hv, a.T, a.B, kC);
     if (e != cudaSuccess) return e;
-    dim3 pgrid((unsigned)nch, a.Hk, a.B);
-    gdn_prefill_prep_kernel<InT><<<pgrid, kPrepThreads, sizeof(PrepSmem), stream>>>(a, ws_kq, ws_rec);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    dim3 sgrid(a.Hv, a.B);
-    gdn_prefill_scan_kernel<InT, OutT><<<sgrid, kScanThreads, scan_smem_bytes<InT>(), stream>>>(v_map, a, ws_kq,
-                                                                                                  ws_rec);
+    dim3 grid(a.Hv, a.B);
+    gdn_prefill_scan_kernel<InT, OutT><<<grid, kScanThreads, scan_smem_bytes<InT>(), stream>>>(
+        v_map, a, ws_kq_of(a, workspace), ws_rec_of(a, workspace));
     return cudaGetLastError();
 }
 
@@ -756,15 +763,24 @@ size_t prefill_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int
     return (size_t)B * Hk * nch * kKQBytes + (size_t)B * Hv * nch * kRecBytes;
 }
 
+cudaError_t launch_prefill_prepare(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
+    return a.in_bf16 ? launch_prep<__nv_bfloat16>(a, workspace, stream) : launch_prep<float>(a, workspace, stream);
+}
+
+cudaError_t launch_prefill_scan(const VerifyArgs& a, void* workspace, cudaStream_t stream) {
+    if (a.in_bf16)
+        return a.out_bf16 ? launch_scan<__nv_bfloat16, __nv_bfloat16>(a, workspace, stream)
+                          : launch_scan<__nv_bfloat16, float>(a, workspace, stream);
+    return a.out_bf16 ? launch_scan<float, __nv_bfloat16>(a, workspace, stream)
+                      : launch_scan<float, float>(a, workspace, stream);
+}
+
 cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
     (void)chunk;
     (void)workspace_bytes;
-    if (a.in_bf16)
-        return a.out_bf16 ? launch_tc_prefill<__nv_bfloat16, __nv_bfloat16>(a, workspace, stream)
-                          : launch_tc_prefill<__nv_bfloat16, float>(a, workspace, stream);
-    return a.out_bf16 ? launch_tc_prefill<float, __nv_bfloat16>(a, workspace, stream)
-                      : launch_tc_prefill<float, float>(a, workspace, stream);
+    cudaError_t e = launch_prefill_prepare(a, workspace, stream);
+    return e == cudaSuccess ? launch_prefill_scan(a, workspace, stream) : e;
 }
 
 }  // namespace gdn

@@ -20,6 +20,12 @@ size_t prefill_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int
 cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+// The two phases launch_prefill runs in order on one stream: the state-independent
+// preparation (normalised keys / queries, per-chunk operators) into the workspace, then the
+// sequential scan over the chunks, which reads it.
+cudaError_t launch_prefill_prepare(const VerifyArgs& a, void* workspace, cudaStream_t stream);
+cudaError_t launch_prefill_scan(const VerifyArgs& a, void* workspace, cudaStream_t stream);
+
 // Size of the fixed device scratch behind gdn_chunk_prefill_noalloc (include/gdn.h).
 constexpr size_t kNoAllocScratchBytes = GDN_NOALLOC_SCRATCH_BYTES;
 

@@ -61,8 +61,10 @@ def _load():
     lib.gdn_decode_step.argtypes = [S] + [_VP] * 10
     lib.gdn_chunk_prefill.argtypes = ([S, ctypes.c_int32] + [_VP] * 11 + [ctypes.c_size_t, _VP])
     lib.gdn_chunk_prefill_noalloc.argtypes = [S, ctypes.c_int32] + [_VP] * 11
+    lib.gdn_chunk_prefill_prepare.argtypes = [S, ctypes.c_int32] + [_VP] * 7 + [ctypes.c_size_t, _VP]
+    lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
     for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill",
-               "gdn_chunk_prefill_noalloc"):
+               "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -203,6 +205,41 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, 
                                      _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state_in),
                                      _ptr(state_out), _ptr(o), _ptr(workspace), wbytes,
                                      _stream(stream)))
+    return o, state_out
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def chunk_prefill_prepare(q, k, a, b, A_log, dt_bias, workspace, H_v=None, d_v=None, chunk=64,
+                          l2_eps=1e-6, scale=1.0, status_word=None, out_dtype=torch.float32,
+                          stream=None):
+    """First phase of chunk_prefill: the state-independent per-chunk operators of the prompt
+    into ``workspace`` (uint8 CUDA tensor of prefill_workspace_bytes()). H_v defaults to
+    a.shape[2], d_v to d_k."""
+    B, T, H_k, d_k = k.shape
+    H_v = a.shape[2] if H_v is None else H_v
+    d_v = d_k if d_v is None else d_v
+    sh = make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
+    _check(_load().gdn_chunk_prefill_prepare(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(a), _ptr(b),
+                                             _ptr(A_log), _ptr(dt_bias), _ptr(workspace),
+                                             _nbytes(workspace), _stream(stream)))
+
+
+def chunk_prefill_scan(v, workspace, H_k, state_in=None, state_out=None, o=None, d_k=None, chunk=64,
+                       status_word=None, out_dtype=torch.float32, stream=None):
+    """Second phase of chunk_prefill: the scan over the chunks of a prepared ``workspace``.
+    Returns (o, state_out); ``H_k`` (and d_k, default d_v) must match the prepare call."""
+    B, T, H_v, d_v = v.shape
+    d_k = d_v if d_k is None else d_k
+    sh = make_shape(B, T, H_k, H_v, d_k, d_v, v.dtype, out_dtype, status_word=status_word)
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    if state_out is None:
+        state_out = torch.empty((B, H_v, d_v, d_k), dtype=torch.float32, device=v.device)
+    _check(_load().gdn_chunk_prefill_scan(ctypes.byref(sh), chunk, _ptr(v), _ptr(state_in), _ptr(state_out),
+                                          _ptr(o), _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return o, state_out
 
 

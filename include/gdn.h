@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2   /* 2: prefill split into prepare / scan; prefill workspace layout */
 
 typedef enum {
     GDN_OK = 0,
@@ -156,6 +156,34 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
                              const float* state_in, float* state_out, void* o,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gdn_chunk_prefill_prepare / gdn_chunk_prefill_scan -- the two phases gdn_chunk_prefill runs
+ * in order on its stream, for callers that schedule them separately (for instance the
+ * preparation of the next prompt alongside the scan of this one, or timing each phase). Same
+ * recurrence and chunk algebra as gdn_chunk_prefill; the split itself has no counterpart in
+ * the source pages.
+ *   prepare  reads q, k [B,T,H_k,d_k], a, b [B,T,H_v], A_log, dt_bias [H_v] and writes every
+ *            per-chunk operator the scan needs into the workspace: the normalised keys and
+ *            queries once per (sequence, key head, chunk), and per (sequence, value head,
+ *            chunk) the decays, the write strengths and the chunk's output / state-update
+ *            operators. No state is read. Chunks are independent and run in parallel.
+ *   scan     reads v [B,T,H_v,d_v], state_in (NULL = zero), the prepared workspace, and writes
+ *            o and state_out exactly as gdn_chunk_prefill does; it walks the chunks in order.
+ * The shape (including H_k, which lays out the workspace), chunk, workspace and
+ * workspace_bytes must be the same in both calls, and the scan must be ordered after the
+ * prepare (same stream, or an event between them). The workspace belongs to the caller and
+ * must not be reused by another call until the scan has completed. Errors are those of
+ * gdn_chunk_prefill (GDN_ERR_WORKSPACE for a missing or short workspace).
+ */
+gdn_status gdn_chunk_prefill_prepare(const gdn_shape* shape, int32_t chunk,
+                                     const void* q, const void* k,
+                                     const void* a, const void* b,
+                                     const float* A_log, const float* dt_bias,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+gdn_status gdn_chunk_prefill_scan(const gdn_shape* shape, int32_t chunk,
+                                  const void* v, const float* state_in, float* state_out, void* o,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the fixed device scratch behind gdn_chunk_prefill_noalloc: 64 MiB. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
@@ -172,8 +200,9 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
  *     allocated until the process exits, whether or not this entry point is called.
  *   - Shapes whose workspace (gdn_chunk_prefill_workspace_bytes) exceeds it are rejected with
  *     GDN_ERR_UNSUPPORTED and a gdn_last_error() message giving both sizes; with d = 128 and
- *     chunk 64 each (sequence, value head, 64-token chunk) needs 49,728 bytes, e.g. up to 28
- *     chunks (1,792 tokens) for B = 1 and H_v = 48.
+ *     chunk 64 each 64-token chunk of a sequence needs 49,728 bytes per value head plus
+ *     65,536 bytes per key head, e.g. up to 19 chunks (1,216 tokens) for B = 1, H_v = 48 and
+ *     H_k = 16.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - All calls on one GPU share the same scratch and it keeps the last call's contents.
  *     Nothing in it needs to start at zero (each call writes every element it later reads),
@@ -192,7 +221,9 @@ gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk,
 /* Bytes of stash gdn_verify_step writes for this shape (0 for an invalid shape). */
 size_t gdn_stash_bytes(const gdn_shape* shape);
 
-/* Bytes of workspace gdn_chunk_prefill needs (0 for an invalid shape or chunk). */
+/* Bytes of workspace gdn_chunk_prefill (and each of its two phases) needs (0 for an invalid
+ * shape or chunk): per sequence and 64-token chunk, 65,536 bytes per key head and 49,728 per
+ * value head. */
 size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk);
 
 /* Static description of a status code. */

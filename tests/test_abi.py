@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 1
+    assert lib.gdn_abi_version() == 2
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -97,3 +97,28 @@ def test_empty_batch_is_a_no_op(gdn):
     sh = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
     assert gdn.lib().gdn_verify_step(ctypes.byref(sh), *([None] * 12), None) == 0
     assert gdn.lib().gdn_commit(ctypes.byref(sh), None, None, None, None, None) == 0
+
+
+def test_prefill_phase_entry_points_validate_on_the_host(gdn):
+    INVALID, UNSUP, WORKSPACE = -1, -2, -4
+    lib = gdn.lib()
+    sh = gdn.make_shape(B=1, T=300, H_k=2, H_v=6, d_k=128, d_v=128)
+    need = gdn.prefill_workspace_bytes(1, 300, 2, 6, 128, 128)
+    # 5 chunks: 2 key heads x 65,536 + 6 value heads x 49,728 bytes per chunk
+    assert need == 5 * (2 * 65536 + 6 * 49728)
+    fake = 0x10000
+    prep = lambda chunk, ws, nbytes, **kw: lib.gdn_chunk_prefill_prepare(
+        ctypes.byref(sh), chunk, kw.get("q", fake), fake, fake, fake, fake, fake, ws, nbytes, None)
+    scan = lambda chunk, ws, nbytes, **kw: lib.gdn_chunk_prefill_scan(
+        ctypes.byref(sh), chunk, kw.get("v", fake), None, fake, fake, ws, nbytes, None)
+    assert prep(64, None, 0) == WORKSPACE
+    assert scan(64, fake, need - 16) == WORKSPACE
+    assert "workspace of %d bytes needed" % need in lib.gdn_last_error().decode()
+    assert prep(32, fake, need) == UNSUP
+    assert scan(64, fake + 8, need) == INVALID                     # misaligned workspace
+    assert prep(64, fake, need, q=None) == INVALID
+    assert "q is NULL" in lib.gdn_last_error().decode()
+    assert scan(64, fake, need, v=None) == INVALID
+    assert "v is NULL" in lib.gdn_last_error().decode()
+    empty = gdn.make_shape(B=0, T=300, H_k=2, H_v=6, d_k=128, d_v=128)
+    assert lib.gdn_chunk_prefill_scan(ctypes.byref(empty), 64, *([None] * 5), 0, None) == 0

@@ -97,3 +97,20 @@ def test_prefill_batch_of_two_grouped_heads(gdn):
     xd = to_dev(x)
     o, S = run_gpu(gdn, xd, xd["S0"])
     assert rel_err(o, o_ref) <= TOL_PREFILL and rel_err(S, S_ref) <= TOL_PREFILL
+
+
+def test_prefill_phases_match_the_one_call_prefill(gdn):
+    # prepare then scan (the two phases gdn_chunk_prefill runs) give the same bits; a second
+    # prompt prepared into its own workspace in between does not disturb the first.
+    w = workload("prefill", T=700, H_k=2, H_v=6, seed=80, state_std=0.05)
+    x = to_dev(make_inputs(w, gates="gentle"))
+    x2 = to_dev(make_inputs(workload("prefill", T=700, H_k=2, H_v=6, seed=81), gates="config"))
+    o_ref, s_ref = run_gpu(gdn, x, x["S0"])
+    nb = gdn.prefill_workspace_bytes(w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    ws2 = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    gdn.chunk_prefill_prepare(x["q"], x["k"], x["a"], x["b"], x["A_log"], x["dt_bias"], ws)
+    gdn.chunk_prefill_prepare(x2["q"], x2["k"], x2["a"], x2["b"], x2["A_log"], x2["dt_bias"], ws2)
+    o, s = gdn.chunk_prefill_scan(x["v"], ws, w.H_k, x["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(s, s_ref)

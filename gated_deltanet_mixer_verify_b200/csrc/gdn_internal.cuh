@@ -28,6 +28,8 @@ struct VerifyArgs {
     int32_t* status_word;
     int always_commit;           // decode: commit all T tokens, ignore accept_len
     int row_split;               // head kernel: CTAs (work items) per head, set by its launcher
+    int prefetch_ahead;          // tensor-core verify: the item whose inputs a CTA prefetches into
+                                 // L2 is its own + this (0: none), set by its launcher
 };
 
 // Arguments of the second phase of a two-phase commit.

@@ -12,9 +12,11 @@
 // Shared memory holds the raw fp32 state tile (TMA, 128-byte swizzle): a kind::tf32 MMA
 // reads a 32-bit container as its truncated tf32 value, so that tile serves directly as S_hi.
 // S_lo = S - S_hi is formed by the threads and stored in tensor memory, where the third pass
-// takes its A operand. That keeps a CTA at ~100 KB of shared memory and 160 tensor-memory
+// takes its A operand. That keeps a CTA at ~100 KB of shared memory and 256 tensor-memory
 // columns, so two CTAs (16 warps) share an SM and overlap one head's copies and algebra with
-// the other's MMAs and commit. One CTA per (sequence, head).
+// the other's MMAs and commit. One CTA per (sequence, head); each CTA also prefetches into L2
+// the inputs of the CTA one resident wave ahead, and splits its state as soon as it lands,
+// while warp 0 is still on the gate chain.
 // Every mbarrier wait is bounded; a timeout sets GDN_STATUS_WAIT_TIMEOUT, suppresses the
 // CTA's global writes, drains its copy and MMAs (bounded) and frees its tensor memory.
 #include <cuda.h>
@@ -48,17 +50,23 @@ struct __align__(1024) TcSmem {
     float Gram[NB][TM];
     float G[TM], Beta[TM], D[TM];
     float A[TM][TM], Cq[TM][TM], Tm[TM][TM], Mo[TM][TM], E[TM][TM];
+    float Ec[TM];            // decay from token t to the last accepted token
     float DL;
     int L;
     int fail;                // a bounded wait ran out
-    uint32_t tmem_d;         // 32 columns: the dots, 128 lanes x 16
-    uint32_t tmem_a;         // 128 columns: S_lo as the A operand of the third pass
+    uint32_t tmem;           // 256 columns: S_lo (A operand of the third pass) at 0..127, the
+                             // dots (128 lanes x 32) at 128..159
     uint64_t full;
     uint64_t mma_done;
 };
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Arrive at named barrier `id` (expecting nthreads) without waiting for it.
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Committed rows for a compile-time number LL of accepted tokens: S_L = d S_0 + sum_{s<LL}
@@ -119,55 +127,68 @@ __global__ void __launch_bounds__(kThreads, 2)
         return;
     }
 
-    // 0. Request the head's state; allocate tensor memory.
-    if (tid == 0) {
+    // 0. Every global load the CTA makes is issued here, before any arithmetic waits on one
+    // (they are dependent round trips otherwise): the 64 KB state tile first, then the small
+    // per-token loads.
+    if (tid == 128) {
         mbar_init(&sm.full, 1);
         mbar_init(&sm.mma_done, 1);
         fence_barrier_init();
         mbar_arrive_expect_tx(&sm.full, kTileBytes);
         for (int kb = 0; kb < 4; ++kb) tc::tma_load_2d(&sm.S[kb * DV * 32], &smap, kb * 32, item * DV, &sm.full);
-        sm.fail = 0;
     }
-    if (warp == 0) {
-        tc::tmem_alloc(&sm.tmem_d, 32);
-        tc::tmem_alloc(&sm.tmem_a, 128);
-        tc::tmem_relinquish();
+    float a_in = 0.f, b_in = 0.f, alog = 0.f, dtb = 0.f;
+    int L_in = 0;
+    if (warp == 0) {   // gate inputs (lane t = token t) and the accept count
+        if (lane < T) {
+            const size_t gi = ((size_t)b * T + lane) * p.Hv + h;
+            a_in = ld_in<InT>(p.a, gi);
+            b_in = ld_in<InT>(p.b, gi);
+        }
+        alog = p.A_log[h];
+        dtb = p.dt_bias[h];
+        if (lane == 0 && !p.always_commit && p.accept_len) L_in = p.accept_len[b];
     }
-
-    // Per-row v_t, fetched early (rows 0..127 belong to threads 0..127).
+    // khat_t, qhat_t (16 lanes per vector, 8 columns per lane) and the per-row v_t (row
+    // tid % 128: threads tid and tid + 128 share a row and split its outputs).
+    const int c16 = tid & 15;
+    const int nrow = tid >> 4;               // 0..15 = NB rows
+    const bool isq = nrow >= TM;
+    const int tq = isq ? nrow - TM : nrow;
+    const bool live = tq < T;
+    float x[8];
+    if (live) {
+        ld8<InT>(isq ? p.q : p.k, (((size_t)b * T + tq) * p.Hk + g) * DK + 8 * c16, x);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    }
     float vrow[TM];
 #pragma unroll
     for (int t = 0; t < TM; ++t)
-        vrow[t] = (tid < DV && t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + tid) : 0.f;
-
-    // 1a. khat_t, qhat_t: 16 lanes per vector, 8 columns per lane; plain copy + split tiles.
-    {
-        const int c16 = tid & 15;
-        const int n = tid >> 4;              // 0..15 = NB rows
-        const bool isq = n >= TM;
-        const int t = isq ? n - TM : n;
-        const bool live = t < T;
-        float x[8];
-        if (live) {
-            ld8<InT>(isq ? p.q : p.k, (((size_t)b * T + t) * p.Hk + g) * DK + 8 * c16, x);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = 0.f;
-        }
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-        ss = group_sum<16>(ss);
-        const float inv = live ? (isq ? p.scale : 1.f) / sqrtf(ss + p.l2_eps) : 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float4 y, hi, lo;
-            y = make_float4(x[4 * half] * inv, x[4 * half + 1] * inv, x[4 * half + 2] * inv, x[4 * half + 3] * inv);
-            hi = make_float4(tc::tf32_hi(y.x), tc::tf32_hi(y.y), tc::tf32_hi(y.z), tc::tf32_hi(y.w));
-            lo = make_float4(y.x - hi.x, y.y - hi.y, y.z - hi.z, y.w - hi.w);
-            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(n, 8 * c16 + 4 * half, 2 * NB) / 4]) = hi;
-            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(NB + n, 8 * c16 + 4 * half, 2 * NB) / 4]) = lo;
-            *reinterpret_cast<float4*>(&sm.KQ[n][8 * c16 + 4 * half]) = y;
+        vrow[t] = (t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + (tid & (DV - 1))) : 0.f;
+    if (warp == 4) {   // tensor memory: one allocation, off the gate chain
+        if (lane == 0) sm.fail = 0;
+        tc::tmem_alloc(&sm.tmem, 256);
+        tc::tmem_relinquish();
+    }
+    // The CTA one resident wave ahead will find its state and per-token inputs in L2: without
+    // this, every CTA starts by waiting on DRAM reads and the SM's two CTAs often wait at the
+    // same time.
+    if (p.prefetch_ahead > 0 && item + p.prefetch_ahead < (int)gridDim.x) {
+        const int nx = item + p.prefetch_ahead;
+        const int nh = nx % p.Hv, nb = nx / p.Hv, ng = nh / (p.Hv / p.Hk);
+        const size_t el = p.in_bf16 ? 2 : 4;
+        // Only whole rows of the state, q, k and v: each lies inside its array.
+        if (tid == 32) bulk_prefetch_l2(p.state_in + (size_t)nx * DV * DK, kTileBytes);
+        if (tid >= 64 && tid < 64 + T) {   // one token of q, k and v per thread
+            const int t = tid - 64;
+            const char* qb = static_cast<const char*>(p.q);
+            const char* kb = static_cast<const char*>(p.k);
+            const char* vb = static_cast<const char*>(p.v);
+            bulk_prefetch_l2(qb + ((((size_t)nb * T + t) * p.Hk + ng) * DK) * el, (uint32_t)(DK * el));
+            bulk_prefetch_l2(kb + ((((size_t)nb * T + t) * p.Hk + ng) * DK) * el, (uint32_t)(DK * el));
+            bulk_prefetch_l2(vb + ((((size_t)nb * T + t) * p.Hv + nh) * DV) * el, (uint32_t)(DV * el));
         }
     }
 
@@ -175,9 +196,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 0) {
         float gl = 0.f, be = 0.f;
         if (lane < T) {
-            const size_t gi = ((size_t)b * T + lane) * p.Hv + h;
-            gl = -expf(p.A_log[h]) * softplus_f(ld_in<InT>(p.a, gi) + p.dt_bias[h]);
-            be = 1.f / (1.f + expf(-ld_in<InT>(p.b, gi)));
+            gl = -expf(alog) * softplus_f(a_in + dtb);
+            be = 1.f / (1.f + expf(-b_in));
         }
         float Gs = gl;
 #pragma unroll
@@ -195,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (p.always_commit) {
                 L = T;
             } else if (p.accept_len) {
-                L = p.accept_len[b];
+                L = L_in;
                 if (L < 0 || L > T) {
                     if (p.status_word && h == 0) atomicOr(p.status_word, kStatusBadAccept);
                     L = -1;
@@ -206,16 +226,64 @@ __global__ void __launch_bounds__(kThreads, 2)
             sm.L = L;
         }
     }
+
+    // 1a. Normalised khat_t, qhat_t: plain copy + the split B tiles of the MMA; each thread
+    // keeps its 8 normalised values for the Gram.
+    float yv[8];
+    {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+        ss = group_sum<16>(ss);
+        const float inv = live ? (isq ? p.scale : 1.f) / sqrtf(ss + p.l2_eps) : 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float4 y, hi, lo;
+            y = make_float4(x[4 * half] * inv, x[4 * half + 1] * inv, x[4 * half + 2] * inv, x[4 * half + 3] * inv);
+            yv[4 * half] = y.x;
+            yv[4 * half + 1] = y.y;
+            yv[4 * half + 2] = y.z;
+            yv[4 * half + 3] = y.w;
+            hi = make_float4(tc::tf32_hi(y.x), tc::tf32_hi(y.y), tc::tf32_hi(y.z), tc::tf32_hi(y.w));
+            lo = make_float4(y.x - hi.x, y.y - hi.y, y.z - hi.z, y.w - hi.w);
+            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(nrow, 8 * c16 + 4 * half, 2 * NB) / 4]) = hi;
+            *reinterpret_cast<float4*>(&sm.B2[tc::sw128_offset(NB + nrow, 8 * c16 + 4 * half, 2 * NB) / 4]) = lo;
+            *reinterpret_cast<float4*>(&sm.KQ[nrow][8 * c16 + 4 * half]) = y;
+        }
+    }
     tc::fence_proxy_async_smem();   // the tensor core will read the B tiles written above
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem_d = sm.tmem_d, tmem_a = sm.tmem_a;
+    const uint32_t tmem_a = sm.tmem, tmem_d = sm.tmem + 128;
+
+    // 2g. Gram rows [Khat; Qhat] Khat^T, all threads, before the split and the MMAs (which
+    // slow it down several-fold when they run alongside): thread (row n, lane c16) dots its 8
+    // normalised columns (registers) with those of each khat_s, the row's 16 lanes reduce them
+    // (halving butterfly), and lane 2s keeps entry s. Warps 4..7 only arrive at barrier 3.
+    {
+        float part[TM];
+#pragma unroll
+        for (int s = 0; s < TM; ++s) {
+            const float4 k0 = *reinterpret_cast<const float4*>(&sm.KQ[s][8 * c16]);
+            const float4 k1 = *reinterpret_cast<const float4*>(&sm.KQ[s][8 * c16 + 4]);
+            float d = yv[0] * k0.x;
+            d = fmaf(yv[1], k0.y, d);
+            d = fmaf(yv[2], k0.z, d);
+            d = fmaf(yv[3], k0.w, d);
+            d = fmaf(yv[4], k1.x, d);
+            d = fmaf(yv[5], k1.y, d);
+            d = fmaf(yv[6], k1.z, d);
+            part[s] = fmaf(yv[7], k1.w, d);
+        }
+        Halve<TM, 8>::run(part, c16);
+        if ((c16 & 1) == 0) sm.Gram[nrow][c16 >> 1] = part[0];
+    }
 
     if (warp >= 4) {
-        // 2s. Warps 4..7: S_lo = S - trunc_tf32(S) into tensor memory (warp w owns lanes
-        // 32 (w - 4) .. +31, i.e. those state rows, all 128 columns), then one thread issues
-        // the three tf32 passes: S (smem) B_hi + S (smem) B_lo + S_lo (tmem) B_hi.
+        named_arrive(3, 256);   // Gram rows 8..15 are stored
+        // 2s. Warps 4..7 (the longest path): S_lo = S - trunc_tf32(S) into tensor memory (warp w owns lanes
+        // 32 (w - 4) .. +31, i.e. those state rows, all 128 columns).
         const int q4 = warp - 4;
         const int row = 32 * q4 + lane;
         if (!mbar_wait_bounded(&sm.full, 0, kMaxPolls)) sm.fail = 1;
@@ -224,18 +292,20 @@ __global__ void __launch_bounds__(kThreads, 2)
             float v[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float4 x = *reinterpret_cast<const float4*>(
+                const float4 xs = *reinterpret_cast<const float4*>(
                     &sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
-                v[4 * q + 0] = x.x - tc::tf32_hi(x.x);
-                v[4 * q + 1] = x.y - tc::tf32_hi(x.y);
-                v[4 * q + 2] = x.z - tc::tf32_hi(x.z);
-                v[4 * q + 3] = x.w - tc::tf32_hi(x.w);
+                v[4 * q + 0] = xs.x - tc::tf32_hi(xs.x);
+                v[4 * q + 1] = xs.y - tc::tf32_hi(xs.y);
+                v[4 * q + 2] = xs.z - tc::tf32_hi(xs.z);
+                v[4 * q + 3] = xs.w - tc::tf32_hi(xs.w);
             }
             tc::tmem_st32(tmem_a + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
         }
         tc::fence_before_sync();
         named_sync(2, 128);
         tc::fence_after_sync();
+        // Then one thread issues the three tf32 passes: S (smem) B_hi + S (smem) B_lo +
+        // S_lo (tmem) B_hi.
         if (tid == 128 && !sm.fail) {
             // Columns 0..15 accumulate S B_hi + S_lo B_hi, columns 16..31 S B_lo.
             const uint32_t id32 = tc::idesc_tf32(DV, 2 * NB), id16 = tc::idesc_tf32(DV, NB);
@@ -256,71 +326,65 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc::mma_commit(&sm.mma_done);
         }
     } else {
-        // 2a. Warps 0..3 meanwhile: Gram rows [Khat; Qhat] Khat^T (8 lanes per row, interleaved
-        // float4 columns, halving butterfly) ...
-        {
-            const int c8 = tid & 7;
-            const int n = tid >> 3;          // 0..15
-            float4 xr[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) xr[m] = *reinterpret_cast<const float4*>(&sm.KQ[n][4 * (c8 + 8 * m)]);
-            float part[TM];
-#pragma unroll
-            for (int s = 0; s < TM; ++s) {
-                float d = 0.f;
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float4 y = *reinterpret_cast<const float4*>(&sm.KQ[s][4 * (c8 + 8 * m)]);
-                    d = fmaf(xr[m].x, y.x, d);
-                    d = fmaf(xr[m].y, y.y, d);
-                    d = fmaf(xr[m].z, y.z, d);
-                    d = fmaf(xr[m].w, y.w, d);
-                }
-                part[s] = d;
-            }
-            Halve<TM, 4>::run(part, c8);
-            sm.Gram[n][c8] = part[0];
+        named_sync(3, 256);     // all 16 Gram rows are stored
+        // ... the T x T algebra (barrier 1 between steps): the decayed coefficients, one entry
+        // per thread, and the commit decays ...
+        const int Lc = sm.L;
+        if (tid < TM * TM) {
+            const int t = tid / TM, s = tid % TM;
+            const bool inq = t < T && s <= t;
+            const float dec = inq ? expf(sm.G[t] - sm.G[s]) : 0.f;
+            sm.A[t][s] = (inq && s < t) ? sm.Beta[t] * dec * sm.Gram[t][s] : 0.f;
+            sm.Cq[t][s] = inq ? dec * sm.Gram[TM + t][s] : 0.f;
+        } else if (tid < TM * TM + TM) {
+            const int t = tid - TM * TM;
+            sm.Ec[t] = (Lc > 0 && t < Lc) ? expf(sm.G[Lc - 1] - sm.G[t]) : 0.f;
         }
         named_sync(1, 128);
-        // ... the decayed coefficients, the triangular inverse, output and commit coefficients
-        // (warp 0) ...
-        if (warp == 0) {
-            for (int e = lane; e < TM * TM; e += 32) {
-                const int t = e / TM, s = e % TM;
-                const bool inq = t < T && s <= t;
-                const float dec = inq ? expf(sm.G[t] - sm.G[s]) : 0.f;
-                sm.A[t][s] = (inq && s < t) ? sm.Beta[t] * dec * sm.Gram[t][s] : 0.f;
-                sm.Cq[t][s] = inq ? dec * sm.Gram[TM + t][s] : 0.f;
-            }
-            __syncwarp();
-            if (lane < TM) {
-                const int s = lane;
-                float col[TM];
+        // ... the unit-triangular inverse Tm = (I + A)^-1 by forward substitution (warp 0, lane
+        // s = column s, A read once into registers) ...
+        if (warp == 0 && lane < TM) {
+            const int s = lane;
+            float a[TM][TM];
 #pragma unroll
-                for (int t = 0; t < TM; ++t) {
-                    float x = (t == s) ? 1.f : 0.f;
+            for (int t = 0; t < TM; ++t)
 #pragma unroll
-                    for (int m = 0; m < t; ++m) x = fmaf(-sm.A[t][m], col[m], x);
-                    col[t] = (t >= s) ? x : 0.f;
-                    sm.Tm[t][s] = col[t];
+                for (int m = 0; m < TM; m += 4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(&sm.A[t][m]);
+                    a[t][m] = v4.x;
+                    a[t][m + 1] = v4.y;
+                    a[t][m + 2] = v4.z;
+                    a[t][m + 3] = v4.w;
                 }
-            }
-            __syncwarp();
-            const int L = sm.L;
-            for (int e = lane; e < TM * TM; e += 32) {
-                const int t = e / TM, s = e % TM;
-                float acc = 0.f;
+            float col[TM];
 #pragma unroll
-                for (int m = 0; m < TM; ++m)
-                    if (m >= s && m <= t) acc = fmaf(sm.Cq[t][m], sm.Tm[m][s], acc);
-                sm.Mo[t][s] = (s <= t) ? acc : 0.f;
-                sm.E[t][s] = (L > 0 && t < L && s <= t) ? expf(sm.G[L - 1] - sm.G[t]) * sm.Tm[t][s] : 0.f;
+            for (int t = 0; t < TM; ++t) {
+                float x = (t == s) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < t; ++m) x = fmaf(-a[t][m], col[m], x);
+                col[t] = (t >= s) ? x : 0.f;
+                sm.Tm[t][s] = col[t];
             }
-            if (lane == 0) sm.DL = (L > 0) ? sm.D[L - 1] : 1.f;
         }
+        named_sync(1, 128);
+        // ... the output and commit coefficients Mo = Cq Tm, E[t][s] = Ec[t] Tm[t][s] (one
+        // entry per thread) ...
+        if (tid < TM * TM) {
+            const int t = tid / TM, s = tid % TM;
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < TM; ++m)
+                if (m >= s && m <= t) acc = fmaf(sm.Cq[t][m], sm.Tm[m][s], acc);
+            sm.Mo[t][s] = (s <= t) ? acc : 0.f;
+        } else {
+            const int e = tid - TM * TM;
+            const int t = e / TM, s = e % TM;
+            sm.E[t][s] = (s <= t) ? sm.Ec[t] * sm.Tm[t][s] : 0.f;
+        }
+        if (tid == 0) sm.DL = (Lc > 0) ? sm.D[Lc - 1] : 1.f;
         named_sync(1, 128);
         // ... and Keff_s = sum_t E[t][s] khat_t (warps 0..3, column j = tid, 8 entries each).
-        if (sm.L > 0) {
+        if (Lc > 0) {
 #pragma unroll
             for (int s = 0; s < TM; ++s) {
                 float acc = 0.f;
@@ -334,31 +398,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int L = sm.L;
     bool ok = !sm.fail;
 
-    // 3. Rows 0..127 (threads 0..127, one row each): the dots from tensor memory, x_s, the
-    // outputs and (two-phase) the stash; warps 4..7 write the stash's keys and decays.
+    // 3. Row tid % 128 (TMEM lane): the dots from tensor memory and x_s (both halves of the
+    // block), then the outputs and stash of tokens 4 half .. +3 (half = tid / 128); threads
+    // 0..127 keep x for the commit.
     if (ok && !mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls)) ok = false;
     tc::fence_after_sync();
-    if (warp < 4) {
+    {
+        const int row = tid & (DV - 1);
+        const int hb = tid >> 7;
         float dots[16], dlo[16];
-        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * warp) << 16), dots);
-        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * warp) << 16) + 16, dlo);
+        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * (warp & 3)) << 16), dots);
+        tc::tmem_ld16(tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + 16, dlo);
 #pragma unroll
         for (int i = 0; i < 16; ++i) dots[i] += dlo[i];
-        const int row = tid;
         float xs[TM];
 #pragma unroll
         for (int s = 0; s < TM; ++s) xs[s] = sm.Beta[s] * (vrow[s] - sm.D[s] * dots[s]);
+        if (hb == 0) {
 #pragma unroll
-        for (int s = 0; s < TM; s += 2)
-            *reinterpret_cast<float4*>(&sm.X2[row][s]) = make_float4(xs[s], xs[s], xs[s + 1], xs[s + 1]);
+            for (int s = 0; s < TM; s += 2)
+                *reinterpret_cast<float4*>(&sm.X2[row][s]) = make_float4(xs[s], xs[s], xs[s + 1], xs[s + 1]);
+        }
         if (ok) {
             OutT* op = reinterpret_cast<OutT*>(p.o);
 #pragma unroll
-            for (int t = 0; t < TM; ++t) {
+            for (int tt = 0; tt < TM / 2; ++tt) {
+                const int t = (TM / 2) * hb + tt;
                 if (t < T) {
-                    float ov = sm.D[t] * dots[TM + t];
+                    float ov = sm.D[t] * (hb ? dots[TM + TM / 2 + tt] : dots[TM + tt]);   // static indices
 #pragma unroll
-                    for (int s = 0; s <= t; ++s) ov = fmaf(sm.Mo[t][s], xs[s], ov);
+                    for (int s = 0; s < TM; ++s)
+                        if (s <= t) ov = fmaf(sm.Mo[t][s], xs[s], ov);
                     st_out<OutT>(op, vo_base + t * tok_stride + row, ov);
                 }
             }
@@ -366,20 +436,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 float* st = p.stash + head * stash_floats_per_head(T, DK, DV);
                 const size_t off_u = (size_t)T * DK + (((size_t)T + 3) & ~size_t(3));
 #pragma unroll
-                for (int t = 0; t < TM; ++t) {
+                for (int tt = 0; tt < TM / 2; ++tt) {
+                    const int t = (TM / 2) * hb + tt;
                     if (t < T) {
                         float u = 0.f;
 #pragma unroll
-                        for (int s = 0; s <= t; ++s) u = fmaf(sm.Tm[t][s], xs[s], u);
+                        for (int s = 0; s < TM; ++s)
+                            if (s <= t) u = fmaf(sm.Tm[t][s], xs[s], u);
                         st[off_u + (size_t)t * DV + row] = u;
                     }
                 }
+                for (int e = tid; e < T * DK; e += kThreads) st[e] = sm.KQ[e / DK][e % DK];
+                if (tid < T) st[(size_t)T * DK + tid] = sm.G[tid];
             }
         }
-    } else if (p.stash && ok) {
-        float* st = p.stash + head * stash_floats_per_head(T, DK, DV);
-        for (int e = tid - 128; e < T * DK; e += 128) st[e] = sm.KQ[e / DK][e % DK];
-        if (tid - 128 < T) st[(size_t)T * DK + (tid - 128)] = sm.G[tid - 128];
     }
     tc::fence_before_sync();
     ok = !__syncthreads_or(!ok);
@@ -409,10 +479,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
-        tc::tmem_dealloc(tmem_a, 128);
-        tc::tmem_dealloc(tmem_d, 32);
-    }
+    if (warp == 4) tc::tmem_dealloc(tmem_a, 256);
 }
 
 template <typename InT, typename OutT>
@@ -428,7 +495,12 @@ cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
     CUtensorMap map;
     cudaError_t e = tc::encode_tmap_f32_sw128(&map, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
     if (e != cudaSuccess) return e;
-    gdn_verify_tc_kernel<InT, OutT><<<a.B * a.Hv, kThreads, smem, stream>>>(map, a);
+    int dev = 0, nsm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    VerifyArgs ap = a;
+    ap.prefetch_ahead = 2 * nsm;   // two CTAs per SM are resident
+    gdn_verify_tc_kernel<InT, OutT><<<a.B * a.Hv, kThreads, smem, stream>>>(map, ap);
     return cudaGetLastError();
 }
 

@@ -170,6 +170,70 @@ gdn_status gdn_commit(const gdn_shape* shape, const float* state_in, float* stat
     return launched(gdn::launch_commit(x, static_cast<cudaStream_t>(stream)), who);
 }
 
+gdn_status gdn_commit_and_verify(const gdn_shape* shape, int32_t prev_T, const void* q, const void* k,
+                                 const void* v, const void* a, const void* b, const float* A_log,
+                                 const float* dt_bias, float* state, const float* prev_stash,
+                                 const int32_t* prev_accept_len, const int32_t* accept_len, void* o,
+                                 float* stash, void* stream) {
+    const char* who = "gdn_commit_and_verify";
+    gdn_status st = check_shape(shape, 16, who);
+    if (st != GDN_OK) return st;
+    if (prev_T < 1 || prev_T > 16) return fail(GDN_ERR_INVALID_ARG, "%s: prev_T = %d not in 1..16", who, (int)prev_T);
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(a, who);
+    REQUIRE_PTR(b, who);
+    REQUIRE_PTR(A_log, who);
+    REQUIRE_PTR(dt_bias, who);
+    REQUIRE_PTR(state, who);
+    REQUIRE_PTR(prev_stash, who);
+    REQUIRE_PTR(prev_accept_len, who);
+    REQUIRE_PTR(o, who);
+    if (accept_len) {
+        REQUIRE_PTR(accept_len, who);
+    } else if (!stash) {
+        return fail(GDN_ERR_INVALID_ARG, "%s: stash is required when accept_len is NULL", who);
+    }
+    if (stash) REQUIRE_PTR(stash, who);
+    gdn::VerifyArgs x = make_args(shape, q, k, v, a, b, A_log, dt_bias);
+    x.state_in = state;
+    x.state_out = state;
+    x.accept_len = accept_len;
+    x.o = o;
+    x.stash = stash;
+    x.always_commit = 0;
+    cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+    int dev = 0, nsm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return launched(e, who);
+    if (gdn::tc_kernel_applies(x, nsm) && prev_T <= 8) {
+        // One pass over the state: the tensor-core kernel applies the previous stash on-chip.
+        x.prev_stash = prev_stash;
+        x.prev_accept_len = prev_accept_len;
+        x.prev_T = prev_T;
+        return launched(gdn::launch_verify(x, s0), who);
+    }
+    // Other shapes: the previous commit in place, then the verify (an extra state pass).
+    gdn::CommitArgs c;
+    c.B = shape->B;
+    c.T = prev_T;
+    c.Hv = shape->H_v;
+    c.dk = shape->d_k;
+    c.dv = shape->d_v;
+    c.state_in = state;
+    c.state_out = state;
+    c.stash = prev_stash;
+    c.accept_len = prev_accept_len;
+    c.status_word = shape->status_word;
+    e = gdn::launch_commit(c, s0);
+    if (e != cudaSuccess) return launched(e, who);
+    if (!accept_len) x.state_out = nullptr;   // two-phase again: the state already holds the new base
+    return launched(gdn::launch_verify(x, s0), who);
+}
+
 gdn_status gdn_decode_step(const gdn_shape* shape, const void* q, const void* k, const void* v,
                            const void* a, const void* b, const float* A_log, const float* dt_bias,
                            float* state, void* o, void* stream) {

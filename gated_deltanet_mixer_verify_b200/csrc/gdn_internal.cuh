@@ -30,6 +30,11 @@ struct VerifyArgs {
     int row_split;               // head kernel: CTAs (work items) per head, set by its launcher
     int prefetch_ahead;          // tensor-core verify: the item whose inputs a CTA prefetches into
                                  // L2 is its own + this (0: none), set by its launcher
+    // Commit-on-next-verify (tensor-core kernel only): the previous two-phase block's stash
+    // (prev_T tokens) and accept counts, applied to state_in before this block (NULL: none).
+    const float* prev_stash;
+    const int32_t* prev_accept_len;
+    int prev_T;
 };
 
 // Arguments of the second phase of a two-phase commit.

@@ -51,6 +51,7 @@ struct __align__(1024) TcSmem {
     float G[TM], Beta[TM], D[TM];
     float A[TM][TM], Cq[TM][TM], Tm[TM][TM], Mo[TM][TM], E[TM][TM];
     float Ec[TM];            // decay from token t to the last accepted token
+    float KP[TM][DK];        // commit-on-next-verify: c_t khat_t of the previous block
     float DL;
     int L;
     int fail;                // a bounded wait ran out
@@ -105,7 +106,8 @@ __device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int wa
     }
 }
 
-template <typename InT, typename OutT>
+// PRE: commit-on-next-verify (the previous block's stash is applied to the state first).
+template <typename InT, typename OutT, bool PRE>
 __global__ void __launch_bounds__(kThreads, 2)
     gdn_verify_tc_kernel(const __grid_constant__ CUtensorMap smap, const VerifyArgs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -167,6 +169,24 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int t = 0; t < TM; ++t)
         vrow[t] = (t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + (tid & (DV - 1))) : 0.f;
+    // Commit-on-next-verify: warps 4..7 load what they need of the previous block's stash
+    // (column j = row i = tid - 128): its accept count and decays, khat_t[j] and u_t[i].
+    constexpr bool precommit = PRE;
+    float kp_raw[TM], up[TM], pG[TM];
+    int pL = 0;
+    if (precommit && warp >= 4) {
+        const int PT = p.prev_T;
+        const int j = tid - 128;
+        const float* st = p.prev_stash + (size_t)item * stash_floats_per_head(PT, DK, DV);
+        const size_t off_u = (size_t)PT * DK + (((size_t)PT + 3) & ~size_t(3));
+        pL = p.prev_accept_len[b];
+#pragma unroll
+        for (int t = 0; t < TM; ++t) {
+            kp_raw[t] = (t < PT) ? st[(size_t)t * DK + j] : 0.f;
+            up[t] = (t < PT) ? st[off_u + (size_t)t * DV + j] : 0.f;
+            pG[t] = (t < PT) ? st[(size_t)PT * DK + t] : 0.f;
+        }
+    }
     if (warp == 4) {   // tensor memory: one allocation, off the gate chain
         if (lane == 0) sm.fail = 0;
         tc::tmem_alloc(&sm.tmem, 256);
@@ -181,6 +201,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const size_t el = p.in_bf16 ? 2 : 4;
         // Only whole rows of the state, q, k and v: each lies inside its array.
         if (tid == 32) bulk_prefetch_l2(p.state_in + (size_t)nx * DV * DK, kTileBytes);
+        if (tid == 33 && p.prev_stash) {
+            const size_t nf = stash_floats_per_head(p.prev_T, DK, DV);   // a multiple of 4 floats
+            bulk_prefetch_l2(p.prev_stash + (size_t)nx * nf, (uint32_t)(nf * sizeof(float)));
+        }
         if (tid >= 64 && tid < 64 + T) {   // one token of q, k and v per thread
             const int t = tid - 64;
             const char* qb = static_cast<const char*>(p.q);
@@ -286,14 +310,39 @@ __global__ void __launch_bounds__(kThreads, 2)
         // 32 (w - 4) .. +31, i.e. those state rows, all 128 columns).
         const int q4 = warp - 4;
         const int row = 32 * q4 + lane;
+        // Commit-on-next-verify: S' = d S + sum_{t < L'} u_t c_t khat_t^T (the previous block
+        // committed at its accept count L'; a bad L' rolls it back and sets status bit 1).
+        // Every thread forms the coefficients; row i = column j = tid - 128 writes c_t khat_t[j].
+        float pdl = 1.f;
+        if (precommit) {
+            int L = pL;
+            if (L < 0 || L > p.prev_T) {
+                if (p.status_word && h == 0 && tid == 128) atomicOr(p.status_word, kStatusBadAccept);
+                L = 0;
+            }
+            float glast = 0.f;
+#pragma unroll
+            for (int t = 0; t < TM; ++t)
+                if (t == L - 1) glast = pG[t];
+            if (L > 0) pdl = expf(glast);
+#pragma unroll
+            for (int t = 0; t < TM; ++t) sm.KP[t][tid - 128] = (t < L) ? expf(glast - pG[t]) * kp_raw[t] : 0.f;
+            named_sync(4, 128);   // KP complete
+        }
         if (!mbar_wait_bounded(&sm.full, 0, kMaxPolls)) sm.fail = 1;
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             float v[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float4 xs = *reinterpret_cast<const float4*>(
-                    &sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
+                float4* sp = reinterpret_cast<float4*>(&sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
+                float4 xs = *sp;
+                if (precommit) {
+                    xs = make_float4(pdl * xs.x, pdl * xs.y, pdl * xs.z, pdl * xs.w);
+#pragma unroll
+                    for (int t = 0; t < TM; ++t) fma4(xs, up[t], *reinterpret_cast<const float4*>(&sm.KP[t][32 * cb + 4 * q]));
+                    *sp = xs;   // S' for the MMAs and the commit
+                }
                 v[4 * q + 0] = xs.x - tc::tf32_hi(xs.x);
                 v[4 * q + 1] = xs.y - tc::tf32_hi(xs.y);
                 v[4 * q + 2] = xs.z - tc::tf32_hi(xs.z);
@@ -301,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tc::tmem_st32(tmem_a + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
         }
+        if (precommit) tc::fence_proxy_async_smem();   // the MMAs read S' written above
         tc::fence_before_sync();
         named_sync(2, 128);
         tc::fence_after_sync();
@@ -456,7 +506,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (!ok && tid == 0 && p.status_word) atomicOr(p.status_word, kStatusWaitTimeout);
 
     // 4. Commit at L (rollback / bad L: the initial state, skipped when in place).
-    if (ok && (L != -2) && !(L <= 0 && p.state_out == p.state_in)) {
+    // After a commit-on-next-verify the state is always written: S' committed at this block's
+    // L, or S' itself (no accept counts: the new base for the next call; rollback; bad L).
+    const bool write_state = precommit || (L != -2 && !(L <= 0 && p.state_out == p.state_in));
+    if (ok && write_state) {
         float* dst = p.state_out + head * (size_t)DV * DK;
         const float dl = sm.DL;
         switch (L > 0 ? L : 0) {
@@ -482,26 +535,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 4) tc::tmem_dealloc(tmem_a, 256);
 }
 
-template <typename InT, typename OutT>
+template <typename InT, typename OutT, bool PRE>
 cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
     constexpr size_t smem = sizeof(TcSmem);
-    static bool configured = false;   // per process; the attribute is per function
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    // Per call: the attribute belongs to the function on the current device.
+    cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT, PRE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     CUtensorMap map;
-    cudaError_t e = tc::encode_tmap_f32_sw128(&map, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
+    e = tc::encode_tmap_f32_sw128(&map, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     VerifyArgs ap = a;
     ap.prefetch_ahead = 2 * nsm;   // two CTAs per SM are resident
-    gdn_verify_tc_kernel<InT, OutT><<<a.B * a.Hv, kThreads, smem, stream>>>(map, ap);
+    gdn_verify_tc_kernel<InT, OutT, PRE><<<a.B * a.Hv, kThreads, smem, stream>>>(map, ap);
     return cudaGetLastError();
+}
+
+template <typename InT, typename OutT>
+cudaError_t launch_tc_pre(const VerifyArgs& a, cudaStream_t stream) {
+    return a.prev_stash ? launch_tc_t<InT, OutT, true>(a, stream) : launch_tc_t<InT, OutT, false>(a, stream);
 }
 
 }  // namespace
@@ -513,9 +569,9 @@ bool tc_kernel_applies(const VerifyArgs& a, int num_sms) {
 
 cudaError_t launch_verify_tc(const VerifyArgs& a, cudaStream_t stream) {
     if (a.in_bf16)
-        return a.out_bf16 ? launch_tc_t<__nv_bfloat16, __nv_bfloat16>(a, stream)
-                          : launch_tc_t<__nv_bfloat16, float>(a, stream);
-    return a.out_bf16 ? launch_tc_t<float, __nv_bfloat16>(a, stream) : launch_tc_t<float, float>(a, stream);
+        return a.out_bf16 ? launch_tc_pre<__nv_bfloat16, __nv_bfloat16>(a, stream)
+                          : launch_tc_pre<__nv_bfloat16, float>(a, stream);
+    return a.out_bf16 ? launch_tc_pre<float, __nv_bfloat16>(a, stream) : launch_tc_pre<float, float>(a, stream);
 }
 
 }  // namespace gdn

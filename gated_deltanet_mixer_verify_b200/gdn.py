@@ -59,11 +59,12 @@ def _load():
     lib.gdn_verify_step.argtypes = [S] + [_VP] * 13
     lib.gdn_commit.argtypes = [S] + [_VP] * 5
     lib.gdn_decode_step.argtypes = [S] + [_VP] * 10
+    lib.gdn_commit_and_verify.argtypes = [S, ctypes.c_int32] + [_VP] * 14
     lib.gdn_chunk_prefill.argtypes = ([S, ctypes.c_int32] + [_VP] * 11 + [ctypes.c_size_t, _VP])
     lib.gdn_chunk_prefill_noalloc.argtypes = [S, ctypes.c_int32] + [_VP] * 11
     lib.gdn_chunk_prefill_prepare.argtypes = [S, ctypes.c_int32] + [_VP] * 7 + [ctypes.c_size_t, _VP]
     lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
-    for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_chunk_prefill",
+    for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_commit_and_verify", "gdn_chunk_prefill",
                "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
@@ -170,6 +171,23 @@ def commit(state_in, stash, accept_len, T, H_k, d_k=None, state_out=None, status
     _check(_load().gdn_commit(ctypes.byref(sh), _ptr(state_in), _ptr(state_out), _ptr(stash),
                               _ptr(accept_len), _stream(stream)))
     return state_out
+
+
+def commit_and_verify(q, k, v, a, b, A_log, dt_bias, state, prev_stash, prev_accept_len, prev_T,
+                      accept_len=None, o=None, stash=None, l2_eps=1e-6, scale=1.0, status_word=None,
+                      out_dtype=torch.float32, stream=None):
+    """Commit-on-next-verify: ``state`` holds the state the previous (two-phase) block started
+    from; its stash and device accept counts are applied on the way in. With ``accept_len``
+    the state ends committed at this block's counts; without it the state ends at the
+    committed previous block and ``stash`` receives this block's. Returns o."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    _check(_load().gdn_commit_and_verify(ctypes.byref(sh), int(prev_T), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                         _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state), _ptr(prev_stash),
+                                         _ptr(prev_accept_len), _ptr(accept_len), _ptr(o), _ptr(stash),
+                                         _stream(stream)))
+    return o
 
 
 def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale=1.0,

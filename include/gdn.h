@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 2   /* 2: prefill split into prepare / scan; prefill workspace layout */
+#define GDN_ABI_VERSION 3   /* 3: gdn_commit_and_verify; 2: prefill split into prepare / scan */
 
 typedef enum {
     GDN_OK = 0,
@@ -137,6 +137,35 @@ gdn_status gdn_decode_step(const gdn_shape* shape,
                            const void* a, const void* b,
                            const float* A_log, const float* dt_bias,
                            float* state, void* o, void* stream);
+
+/*
+ * gdn_commit_and_verify -- commit-on-next-verify: the previous block's two-phase commit is
+ * folded into the next verify block, so that the state is read once and written once per
+ * block even when the accept count is not known at verify time. Passages: the GPU-resident
+ * commit / rollback ("Lithos-metal: Qwen3.8-27B on 40-core M5 Max", runtime paragraph) and
+ * the rewind after every acceptance decision ("Qwen 3.8 27B mac m5: 200 tok/s, audited",
+ * section "How does DSpark speculative decoding create more than one token per read?").
+ *   shape            this block's shape (T tokens).
+ *   prev_T           the previous block's T (1..16): the layout of prev_stash.
+ *   state            in: the state the previous block started from (what that block's
+ *                    gdn_verify_step read); out: see accept_len. [B][H_v][d_v][d_k] fp32.
+ *   prev_stash       what that gdn_verify_step wrote as its stash (two-phase, accept_len NULL).
+ *   prev_accept_len  [B] int32, device: that block's accept counts (0..prev_T; out of range
+ *                    rolls the sequence back to its start and sets status bit 1).
+ *   accept_len       this block's accept counts (device) or NULL:
+ *                    given: state <- this block committed at accept_len (both commits applied);
+ *                    NULL:  state <- the previous block committed at prev_accept_len (the new
+ *                           base), and stash <- this block's stash, for the next call.
+ *   o, stash         as gdn_verify_step; this block's outputs see the committed previous state.
+ * With d_k = d_v = 128, 2 <= T <= 8, prev_T <= 8 and B * H_v at least the SM count, one kernel
+ * does all of it; other shapes run gdn_commit's kernel in place first (one more state pass).
+ */
+gdn_status gdn_commit_and_verify(const gdn_shape* shape, int32_t prev_T,
+                                 const void* q, const void* k, const void* v,
+                                 const void* a, const void* b,
+                                 const float* A_log, const float* dt_bias,
+                                 float* state, const float* prev_stash, const int32_t* prev_accept_len,
+                                 const int32_t* accept_len, void* o, float* stash, void* stream);
 
 /*
  * gdn_chunk_prefill -- the mixer over a long prompt (T tokens per sequence), in the

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 2
+    assert lib.gdn_abi_version() == 3
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -122,3 +122,22 @@ def test_prefill_phase_entry_points_validate_on_the_host(gdn):
     assert "v is NULL" in lib.gdn_last_error().decode()
     empty = gdn.make_shape(B=0, T=300, H_k=2, H_v=6, d_k=128, d_v=128)
     assert lib.gdn_chunk_prefill_scan(ctypes.byref(empty), 64, *([None] * 5), 0, None) == 0
+
+
+def test_commit_and_verify_validates_on_the_host(gdn):
+    INVALID, UNSUP = -1, -2
+    lib = gdn.lib()
+    fake = 0x10000
+    sh = gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    call = lambda prev_T, **kw: lib.gdn_commit_and_verify(
+        ctypes.byref(kw.get("shape", sh)), prev_T, *([fake] * 7), kw.get("state", fake), kw.get("prev_stash", fake),
+        kw.get("prev_L", fake), kw.get("L", fake), fake, kw.get("stash", fake), None)
+    assert call(0) == INVALID and "prev_T" in lib.gdn_last_error().decode()
+    assert call(17) == INVALID
+    assert call(8, prev_stash=None) == INVALID and "prev_stash is NULL" in lib.gdn_last_error().decode()
+    assert call(8, prev_L=None) == INVALID
+    assert call(8, state=None) == INVALID
+    assert call(8, L=None, stash=None) == INVALID and "stash is required" in lib.gdn_last_error().decode()
+    assert call(8, shape=gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=96, d_v=128)) == UNSUP
+    empty = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    assert lib.gdn_commit_and_verify(ctypes.byref(empty), 8, *([None] * 13), None) == 0

@@ -47,18 +47,26 @@ struct __align__(1024) TcSmem {
     float KQ[NB][DK];        // khat, qhat in plain fp32 (Gram, Keff, stash)
     float Keff[TM][DK];
     float2 X2[DV][TM];       // (x_s, x_s) per state row: ready-made operands of the packed FMAs
+    // Commit-on-next-verify: the previous block's stash for this head as stored (khat'_t rows,
+    // scaled in place to KP_t = c_t khat'_t; the decays G'; the u'_t rows), and W = KP [khat;
+    // qhat]^T, the correction of the dots for the committed state.
+    float PS[2 * TM * DK + TM];
+    float W[TM][NB];
     float Gram[NB][TM];
     float G[TM], Beta[TM], D[TM];
     float A[TM][TM], Cq[TM][TM], Tm[TM][TM], Mo[TM][TM], E[TM][TM];
     float Ec[TM];            // decay from token t to the last accepted token
-    float KP[TM][DK];        // commit-on-next-verify: c_t khat_t of the previous block
     float DL;
+    float PD;                // decay of the previous block at its accept count L'
     int L;
-    int fail;                // a bounded wait ran out
+    int PL;                  // L' (0 for an out-of-range count)
+    int fail;                // the state copy's bounded wait ran out
+    int pfail;               // the previous stash copy's bounded wait ran out
     uint32_t tmem;           // 256 columns: S_lo (A operand of the third pass) at 0..127, the
                              // dots (128 lanes x 32) at 128..159
     uint64_t full;
     uint64_t mma_done;
+    uint64_t prev_full;      // the previous stash has landed in PS
 };
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
@@ -72,13 +80,22 @@ __device__ __forceinline__ void named_arrive(int id, int nthreads) {
 
 // Committed rows for a compile-time number LL of accepted tokens: S_L = d S_0 + sum_{s<LL}
 // x_s Keff_s (LL = 0: S_0 unchanged). One warp per 16 rows, a lane per 16-byte column chunk.
-template <int LL>
-__device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int warp, int lane, float dl) {
+// PRE: S_0 is first replaced by the previous block committed at its count L' = Lp,
+// S' = pd S_0 + sum_{t<Lp} u'_t KP_t^T (stash rows in PS, u' rows from offset off_u).
+template <int LL, bool PRE>
+__device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int warp, int lane, float dl, int Lp,
+                                            float pd, int off_u) {
     const int chunk = lane;   // columns 4*chunk .. +3
     const int kb = chunk >> 3, c = chunk & 7;
     float4 ke[LL > 0 ? LL : 1];
 #pragma unroll
     for (int s = 0; s < LL; ++s) ke[s] = *reinterpret_cast<const float4*>(&sm.Keff[s][4 * chunk]);
+    float4 kp[PRE ? TM : 1];
+    if (PRE) {
+#pragma unroll
+        for (int t = 0; t < TM; ++t)
+            kp[t] = (t < Lp) ? *reinterpret_cast<const float4*>(&sm.PS[t * DK + 4 * chunk]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     const float2 dl2 = make_float2(dl, dl);
 #pragma unroll 4
     for (int i = 0; i < DV / 8; ++i) {
@@ -86,6 +103,20 @@ __device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int wa
         const float4 sv =
             *reinterpret_cast<const float4*>(&sm.S[(kb * DV * 128 + row * 128 + ((c ^ (row & 7)) << 4)) / 4]);
         float2 r0 = make_float2(sv.x, sv.y), r1 = make_float2(sv.z, sv.w);
+        if (PRE) {
+            const float2 pd2 = make_float2(pd, pd);
+            r0 = __fmul2_rn(r0, pd2);
+            r1 = __fmul2_rn(r1, pd2);
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                if (t < Lp) {
+                    const float u = sm.PS[off_u + t * DV + row];   // the same word for the whole warp
+                    const float2 u2 = make_float2(u, u);
+                    r0 = __ffma2_rn(u2, make_float2(kp[t].x, kp[t].y), r0);
+                    r1 = __ffma2_rn(u2, make_float2(kp[t].z, kp[t].w), r1);
+                }
+            }
+        }
         if (LL > 0) {
             r0 = __fmul2_rn(r0, dl2);
             r1 = __fmul2_rn(r1, dl2);
@@ -132,16 +163,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 0. Every global load the CTA makes is issued here, before any arithmetic waits on one
     // (they are dependent round trips otherwise): the 64 KB state tile first, then the small
     // per-token loads.
+    // Commit-on-next-verify: the previous block's stash for this head (one bulk copy, beside
+    // the state tile) and its accept count L'.
+    constexpr bool precommit = PRE;
     if (tid == 128) {
         mbar_init(&sm.full, 1);
         mbar_init(&sm.mma_done, 1);
+        if (precommit) mbar_init(&sm.prev_full, 1);
         fence_barrier_init();
         mbar_arrive_expect_tx(&sm.full, kTileBytes);
         for (int kb = 0; kb < 4; ++kb) tc::tma_load_2d(&sm.S[kb * DV * 32], &smap, kb * 32, item * DV, &sm.full);
+        if (precommit) {
+            const size_t nf = stash_floats_per_head(p.prev_T, DK, DV);   // a multiple of 4 floats
+            mbar_arrive_expect_tx(&sm.prev_full, (uint32_t)(nf * sizeof(float)));
+            bulk_g2s(sm.PS, p.prev_stash + (size_t)item * nf, (uint32_t)(nf * sizeof(float)), &sm.prev_full);
+        }
     }
     float a_in = 0.f, b_in = 0.f, alog = 0.f, dtb = 0.f;
-    int L_in = 0;
-    if (warp == 0) {   // gate inputs (lane t = token t) and the accept count
+    int L_in = 0, Lp_in = 0;
+    if (warp == 0) {   // gate inputs (lane t = token t) and the accept counts
         if (lane < T) {
             const size_t gi = ((size_t)b * T + lane) * p.Hv + h;
             a_in = ld_in<InT>(p.a, gi);
@@ -150,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         alog = p.A_log[h];
         dtb = p.dt_bias[h];
         if (lane == 0 && !p.always_commit && p.accept_len) L_in = p.accept_len[b];
+        if (precommit && lane == 1) Lp_in = p.prev_accept_len[b];
     }
     // khat_t, qhat_t (16 lanes per vector, 8 columns per lane) and the per-row v_t (row
     // tid % 128: threads tid and tid + 128 share a row and split its outputs).
@@ -169,26 +210,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int t = 0; t < TM; ++t)
         vrow[t] = (t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + (tid & (DV - 1))) : 0.f;
-    // Commit-on-next-verify: warps 4..7 load what they need of the previous block's stash
-    // (column j = row i = tid - 128): its accept count and decays, khat_t[j] and u_t[i].
-    constexpr bool precommit = PRE;
-    float kp_raw[TM], up[TM], pG[TM];
-    int pL = 0;
-    if (precommit && warp >= 4) {
-        const int PT = p.prev_T;
-        const int j = tid - 128;
-        const float* st = p.prev_stash + (size_t)item * stash_floats_per_head(PT, DK, DV);
-        const size_t off_u = (size_t)PT * DK + (((size_t)PT + 3) & ~size_t(3));
-        pL = p.prev_accept_len[b];
-#pragma unroll
-        for (int t = 0; t < TM; ++t) {
-            kp_raw[t] = (t < PT) ? st[(size_t)t * DK + j] : 0.f;
-            up[t] = (t < PT) ? st[off_u + (size_t)t * DV + j] : 0.f;
-            pG[t] = (t < PT) ? st[(size_t)PT * DK + t] : 0.f;
-        }
-    }
     if (warp == 4) {   // tensor memory: one allocation, off the gate chain
-        if (lane == 0) sm.fail = 0;
+        if (lane == 0) {
+            sm.fail = 0;
+            sm.pfail = 0;
+        }
         tc::tmem_alloc(&sm.tmem, 256);
         tc::tmem_relinquish();
     }
@@ -248,6 +274,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 L = -2;
             }
             sm.L = L;
+        }
+        if (precommit && lane == 1) {
+            int Lp = Lp_in;
+            if (Lp < 0 || Lp > p.prev_T) {
+                if (p.status_word && h == 0) atomicOr(p.status_word, kStatusBadAccept);
+                Lp = 0;
+            }
+            sm.PL = Lp;
         }
     }
 
@@ -310,39 +344,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         // 32 (w - 4) .. +31, i.e. those state rows, all 128 columns).
         const int q4 = warp - 4;
         const int row = 32 * q4 + lane;
-        // Commit-on-next-verify: S' = d S + sum_{t < L'} u_t c_t khat_t^T (the previous block
-        // committed at its accept count L'; a bad L' rolls it back and sets status bit 1).
-        // Every thread forms the coefficients; row i = column j = tid - 128 writes c_t khat_t[j].
-        float pdl = 1.f;
-        if (precommit) {
-            int L = pL;
-            if (L < 0 || L > p.prev_T) {
-                if (p.status_word && h == 0 && tid == 128) atomicOr(p.status_word, kStatusBadAccept);
-                L = 0;
-            }
-            float glast = 0.f;
-#pragma unroll
-            for (int t = 0; t < TM; ++t)
-                if (t == L - 1) glast = pG[t];
-            if (L > 0) pdl = expf(glast);
-#pragma unroll
-            for (int t = 0; t < TM; ++t) sm.KP[t][tid - 128] = (t < L) ? expf(glast - pG[t]) * kp_raw[t] : 0.f;
-            named_sync(4, 128);   // KP complete
-        }
         if (!mbar_wait_bounded(&sm.full, 0, kMaxPolls)) sm.fail = 1;
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             float v[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                float4* sp = reinterpret_cast<float4*>(&sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
-                float4 xs = *sp;
-                if (precommit) {
-                    xs = make_float4(pdl * xs.x, pdl * xs.y, pdl * xs.z, pdl * xs.w);
-#pragma unroll
-                    for (int t = 0; t < TM; ++t) fma4(xs, up[t], *reinterpret_cast<const float4*>(&sm.KP[t][32 * cb + 4 * q]));
-                    *sp = xs;   // S' for the MMAs and the commit
-                }
+                const float4 xs =
+                    *reinterpret_cast<const float4*>(&sm.S[(cb * DV * 128 + row * 128 + ((q ^ (row & 7)) << 4)) / 4]);
                 v[4 * q + 0] = xs.x - tc::tf32_hi(xs.x);
                 v[4 * q + 1] = xs.y - tc::tf32_hi(xs.y);
                 v[4 * q + 2] = xs.z - tc::tf32_hi(xs.z);
@@ -350,7 +359,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tc::tmem_st32(tmem_a + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
         }
-        if (precommit) tc::fence_proxy_async_smem();   // the MMAs read S' written above
         tc::fence_before_sync();
         named_sync(2, 128);
         tc::fence_after_sync();
@@ -380,6 +388,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ... the T x T algebra (barrier 1 between steps): the decayed coefficients, one entry
         // per thread, and the commit decays ...
         const int Lc = sm.L;
+        if (precommit) {
+            if (!mbar_wait_bounded(&sm.prev_full, 0, kMaxPolls)) sm.pfail = 1;
+            const int Lp = sm.PL;
+            const float* pg = &sm.PS[p.prev_T * DK];   // the previous block's cumulative log-decays
+            const float glast = (Lp > 0) ? pg[Lp - 1] : 0.f;
+#pragma unroll
+            for (int t = 0; t < TM; ++t)
+                if (t < Lp) sm.PS[t * DK + tid] *= expf(glast - pg[t]);
+            if (tid == 0) sm.PD = (Lp > 0) ? expf(glast) : 1.f;
+        }
         if (tid < TM * TM) {
             const int t = tid / TM, s = tid % TM;
             const bool inq = t < T && s <= t;
@@ -443,10 +461,30 @@ __global__ void __launch_bounds__(kThreads, 2)
                 sm.Keff[s][tid] = acc;
             }
         }
+        if (precommit) {
+            // ... and W[t][n] = KP_t . [khat; qhat]_n (one entry per thread; rotated columns, so
+            // the 8 threads of a quarter-warp read 8 different bank groups).
+            const int t = tid >> 4, n = tid & (NB - 1);
+            float acc = 0.f;
+            if (t < sm.PL) {
+#pragma unroll 8
+                for (int c = 0; c < DK / 4; ++c) {
+                    const int cc = (c + n) & (DK / 4 - 1);
+                    const float4 kp = *reinterpret_cast<const float4*>(&sm.PS[t * DK + 4 * cc]);
+                    const float4 kq = *reinterpret_cast<const float4*>(&sm.KQ[n][4 * cc]);
+                    acc = fmaf(kp.x, kq.x, acc);
+                    acc = fmaf(kp.y, kq.y, acc);
+                    acc = fmaf(kp.z, kq.z, acc);
+                    acc = fmaf(kp.w, kq.w, acc);
+                }
+            }
+            sm.W[t][n] = acc;
+        }
     }
     __syncthreads();
     const int L = sm.L;
-    bool ok = !sm.fail;
+    bool ok = !sm.fail && !sm.pfail;
+    const int off_pu = p.prev_T * DK + ((p.prev_T + 3) & ~3);   // u' rows in PS
 
     // 3. Row tid % 128 (TMEM lane): the dots from tensor memory and x_s (both halves of the
     // block), then the outputs and stash of tokens 4 half .. +3 (half = tid / 128); threads
@@ -461,6 +499,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc::tmem_ld16(tmem_d + ((uint32_t)(32 * (warp & 3)) << 16) + 16, dlo);
 #pragma unroll
         for (int i = 0; i < 16; ++i) dots[i] += dlo[i];
+        if (precommit) {
+            const float pd = sm.PD;
+            const int Lp = sm.PL;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dots[i] *= pd;
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                if (t < Lp) {
+                    const float u = sm.PS[off_pu + t * DV + row];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dots[i] = fmaf(u, sm.W[t][i], dots[i]);
+                }
+            }
+        }
         float xs[TM];
 #pragma unroll
         for (int s = 0; s < TM; ++s) xs[s] = sm.Beta[s] * (vrow[s] - sm.D[s] * dots[s]);
@@ -512,22 +564,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok && write_state) {
         float* dst = p.state_out + head * (size_t)DV * DK;
         const float dl = sm.DL;
+        const int Lp = precommit ? sm.PL : 0;
+        const float pd = precommit ? sm.PD : 1.f;
         switch (L > 0 ? L : 0) {
-            case 1: commit_rows<1>(sm, dst, warp, lane, dl); break;
-            case 2: commit_rows<2>(sm, dst, warp, lane, dl); break;
-            case 3: commit_rows<3>(sm, dst, warp, lane, dl); break;
-            case 4: commit_rows<4>(sm, dst, warp, lane, dl); break;
-            case 5: commit_rows<5>(sm, dst, warp, lane, dl); break;
-            case 6: commit_rows<6>(sm, dst, warp, lane, dl); break;
-            case 7: commit_rows<7>(sm, dst, warp, lane, dl); break;
-            case 8: commit_rows<8>(sm, dst, warp, lane, dl); break;
-            default: commit_rows<0>(sm, dst, warp, lane, dl); break;
+            case 1: commit_rows<1, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 2: commit_rows<2, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 3: commit_rows<3, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 4: commit_rows<4, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 5: commit_rows<5, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 6: commit_rows<6, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 7: commit_rows<7, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            case 8: commit_rows<8, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
+            default: commit_rows<0, PRE>(sm, dst, warp, lane, dl, Lp, pd, off_pu); break;
         }
     }
 
     // Drain after a timeout (bounded), then free the tensor memory (always).
     if (!ok && tid == 0) {
         mbar_wait_bounded(&sm.full, 0, kMaxPolls);
+        if (precommit) mbar_wait_bounded(&sm.prev_full, 0, kMaxPolls);
         if (!sm.fail) mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls);
     }
     tc::fence_before_sync();

@@ -41,6 +41,7 @@ _CSRC = "gated_deltanet_mixer_verify_b200/csrc/"
 _HEADERS = [_CSRC + f for f in ("gdn_tc.cuh", "gdn_device.cuh", "gdn_internal.cuh")]
 KERNEL_SOURCES = {
     "batched_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
+    "commit_next_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
@@ -147,8 +148,31 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workloads
 
+def stash_floats_per_head(T, dk, dv):
+    """Floats of one (sequence, value head) stash: khat [T][d_k], G [T] and u [T][d_v], the
+    last two padded to a multiple of 4."""
+    pad = lambda n: (n + 3) // 4 * 4
+    return T * dk + pad(T) + pad(T * dv)
+
+
+def commit_next_bytes(w):
+    """Bytes one commit-on-next-verify call must move: the verify call's (the state written
+    back for every sequence) plus the previous block's stash read and this block's written."""
+    stash = w.B * w.H_v * stash_floats_per_head(w.T, w.d_k, w.d_v) * 4
+    return algorithmic_bytes(w, n_state_writes=w.B) + 2 * stash
+
+
 def workload_config(name):
     """The JSON `config` of a workload (what it is, with its sizes)."""
+    if name == "commit_next_verify":
+        c = workload_config("batched_verify")
+        w = workload("batched_verify")
+        c.update(workload=name, accept_len="the previous block's: min(Geometric(0.25), 8) per "
+                 "sequence, device int32",
+                 state="fp32 [B,H_v,d_v,d_k]: the previous block committed in place, this "
+                 "block's stash written (two-phase)",
+                 l2="inputs larger than L2 (%.0f MB moved per step, L2 126 MB)" % (commit_next_bytes(w) / 1e6))
+        return c
     w = workload(name)
     c = {"workload": w.name, "B": w.B, "T": w.T, "H_k": w.H_k, "H_v": w.H_v, "d_k": w.d_k,
          "d_v": w.d_v, "layers": w.layers, "in_dtype": w.in_dtype}
@@ -203,6 +227,35 @@ class Verify:
 
     def per_step_inputs(self):
         return ["q", "k", "v", "a", "b"] + ([] if self.decode else ["accept_len"])
+
+
+class CommitNext(Verify):
+    """commit_next_verify: the serving loop's form of a verify step. Each call applies the
+    previous block's stash at its accept counts (known by now) and verifies the next block on
+    the committed state, writing that block's stash for the next call; two stash buffers
+    alternate."""
+
+    def __init__(self, name, rank, dev):
+        super().__init__("batched_verify", rank, dev)
+        w = self.w
+        n = w.B * w.H_v * stash_floats_per_head(w.T, w.d_k, w.d_v)
+        self.stash = [torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(2)]
+        x = self.x
+        self.gdn.verify_step(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                             self.state, None, None, self.o, stash=self.stash[0])
+        self.k = 0
+        self.bytes = commit_next_bytes(w)
+
+    def step(self, x=None, o=None):
+        x = x or self.x
+        o = self.o if o is None else o
+        prev, cur = self.stash[self.k & 1], self.stash[(self.k + 1) & 1]
+        self.gdn.commit_and_verify(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                                   self.state, prev, x["accept_len"], self.w.T, o=o, stash=cur)
+        self.k += 1
+
+    def config(self):
+        return workload_config("commit_next_verify")
 
 
 class SingleSeq:
@@ -298,7 +351,7 @@ class Prefill:
 
 
 WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
-             "prefill": Prefill}
+             "prefill": Prefill, "commit_next_verify": CommitNext}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -308,7 +361,8 @@ def oracle_sample(name, budget_s, rank=0):
     Returns (seconds per unit, units timed, description, threads)."""
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    w = workload(name, seed=rank_seed(workload(name).seed, rank))
+    shape = "batched_verify" if name == "commit_next_verify" else name
+    w = workload(shape, seed=rank_seed(workload(shape).seed, rank))
     threads = orc.max_threads()
     if name == "prefill":
         sub = workload(name, T=2048, H_k=1, H_v=3)
@@ -319,8 +373,8 @@ def oracle_sample(name, budget_s, rank=0):
         # units are tokens of all 48 heads: 3 of 48 heads timed over 2048 tokens
         per_token = dt / 2048 * (w.H_v / 3)
         return per_token, 2048, "2048 tokens x 3 of 48 value heads (fp64 recurrence)", threads
-    n_seq = {"batched_verify": 8, "decode": 64, "single_seq_verify": 1}[name]
-    sub = workload(name, B=n_seq)
+    n_seq = {"batched_verify": 8, "decode": 64, "single_seq_verify": 1, "commit_next_verify": 8}[name]
+    sub = workload(shape, B=n_seq)
     f = as_f64(make_inputs(sub))
     L = f["accept_len"] if name != "decode" else None
     reps, t_total = 0, 0.0
@@ -333,15 +387,19 @@ def oracle_sample(name, budget_s, rank=0):
             break
     per_seq = t_total / (reps * n_seq)
     desc = "%d sequence(s) x %d value heads x T=%d, %d repetition(s)" % (n_seq, w.H_v, w.T, reps)
+    if name == "commit_next_verify":
+        desc += " (one block verified and committed at its counts per sequence per step)"
     return per_seq, n_seq * reps, desc, threads
 
 
 def cpu_value(name, per_unit_s):
     """The workload metric (GB/s or tok/s) the oracle reaches at per_unit_s per unit."""
-    w = workload(name)
     if name == "prefill":
         return 1.0 / per_unit_s, "tok/s"
-    per_seq_bytes = algorithmic_bytes(workload(name, B=1))
+    if name == "commit_next_verify":
+        per_seq_bytes = commit_next_bytes(workload("batched_verify", B=1))
+    else:
+        per_seq_bytes = algorithmic_bytes(workload(name, B=1))
     return per_seq_bytes / per_unit_s / 1e9, "GB/s"
 
 
@@ -365,13 +423,17 @@ def run_reference(args, rank, world):
         desc = "256 tokens x 3 of 48 value heads per step (fp64 recurrence)"
     else:
         n_seq = 16 if name == "decode" else 1
-        sub = workload(name, B=n_seq)
+        shape = "batched_verify" if name == "commit_next_verify" else name
+        sub = workload(shape, B=n_seq)
         f = as_f64(make_inputs(sub))
         L = None if name == "decode" else f["accept_len"]
         run = lambda: orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
                                  f["dt_bias"], f["S0"], L)
-        units_per_step = algorithmic_bytes(sub) / 1e9          # GB of the workload per step
+        per_step = commit_next_bytes(sub) if name == "commit_next_verify" else algorithmic_bytes(sub)
+        units_per_step = per_step / 1e9                        # GB of the workload per step
         desc = "%d sequence(s) x 48 value heads x T=%d per step" % (n_seq, sub.T)
+        if name == "commit_next_verify":
+            desc += " (one block verified and committed at its counts)"
     for _ in range(args.warmup):
         run()
     t0 = time.perf_counter()

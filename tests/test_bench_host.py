@@ -1,0 +1,52 @@
+"""bench.py's host-side accounting, without a GPU: the stash size it charges matches the
+library's own gdn_stash_bytes, the commit-on-next-verify byte count adds exactly the two
+stashes and the state write-back of every sequence, and the reference arm (the oracle on the
+host cores) prints one JSON line for the new workload."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+from gated_deltanet_mixer_verify_b200 import build as gbuild
+from gated_deltanet_mixer_verify_b200.inputs import workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("T", [1, 5, 8])
+def test_stash_floats_match_the_library(bench, T):
+    gbuild.build()
+    from gated_deltanet_mixer_verify_b200 import gdn
+    assert bench.stash_floats_per_head(T, 128, 128) * 4 * 64 * 48 == gdn.stash_bytes(64, T, 16, 48, 128, 128)
+
+
+def test_commit_next_bytes(bench):
+    w = workload("batched_verify")
+    state = w.B * w.H_v * w.d_v * w.d_k * 4
+    stash = w.B * w.H_v * (w.T * w.d_k + 8 + w.T * w.d_v) * 4
+    # the verify call's bytes with every sequence's state written back, plus two stashes
+    assert bench.commit_next_bytes(w) == bench.algorithmic_bytes(w, n_state_writes=w.B) + 2 * stash
+    assert bench.algorithmic_bytes(w, n_state_writes=w.B) - bench.algorithmic_bytes(w, n_state_writes=0) == state
+
+
+def test_reference_arm_commit_next_verify():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "commit_next_verify", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["config"]["workload"] == "commit_next_verify"
+    assert d["unit"] == "GB/s" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0

@@ -44,6 +44,8 @@ def _load():
         lib.oracle_verify.restype = ctypes.c_int
         lib.oracle_chunked.argtypes = [ctypes.c_int] * 7 + [_D] * 6 + [_D, _D, ctypes.c_int]
         lib.oracle_chunked.restype = ctypes.c_int
+        lib.oracle_short_conv.argtypes = [ctypes.c_int] * 4 + [_D] * 3 + [_I32, _D, _D]
+        lib.oracle_short_conv.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -160,3 +162,41 @@ def prefill(q, k, v, a, b, A_log, dt_bias, S0=None, l2_eps=1e-6, scale=1.0, nthr
         S0 = np.zeros((B, Hv, dv, dk))
     o, Sf, _ = verify(q, k, v, a, b, A_log, dt_bias, S0, None, l2_eps, scale, nthreads)
     return o, Sf
+
+
+def short_conv_channels(x, w, hist, accept_len=None, write_history=True):
+    """Causal short convolution per channel with its rewound history (oracle_short_conv).
+
+    x: [B, T, C]; w: [C, K]; hist: [B, K-1, C] (oldest first); accept_len: [B] or None (all T).
+    Returns (y [B, T, C], new history [B, K-1, C] or None, number of out-of-range counts).
+    """
+    x, w, hist = _f64(x), _f64(w), _f64(hist)
+    B, T, C = x.shape
+    K = w.shape[1]
+    if w.shape[0] != C or hist.shape != (B, K - 1, C):
+        raise ValueError("short_conv: inconsistent shape")
+    y = np.zeros((B, T, C))
+    h_out = np.zeros((B, K - 1, C)) if write_history else None
+    L = None if accept_len is None else np.ascontiguousarray(accept_len, dtype=np.int32)
+    bad = _load().oracle_short_conv(B, T, C, K, _p(x), _p(w), _p(hist), _pi(L), _p(y), _p(h_out))
+    return y, h_out, int(bad)
+
+
+def conv_channels(q, k, v):
+    """Pack q, k [B, T, H_k, d_k] and v [B, T, H_v, d_v] into the channel order of the
+    short convolution: [q heads | k heads | v heads], i.e. [B, T, 2 H_k d_k + H_v d_v]."""
+    B, T = v.shape[0], v.shape[1]
+    return np.concatenate([_f64(q).reshape(B, T, -1), _f64(k).reshape(B, T, -1),
+                           _f64(v).reshape(B, T, -1)], axis=2)
+
+
+def short_conv(q, k, v, w, hist, accept_len=None, write_history=True):
+    """The short convolution applied to the mixer's q, k, v (channel order q | k | v).
+
+    q, k: [B, T, H_k, d_k]; v: [B, T, H_v, d_v]; w: [C, K]; hist: [B, K-1, C].
+    Returns (q', k', v', new history, number of out-of-range counts).
+    """
+    y, h_out, bad = short_conv_channels(conv_channels(q, k, v), w, hist, accept_len, write_history)
+    nq, nk = int(np.prod(q.shape[2:])), int(np.prod(k.shape[2:]))
+    return (y[:, :, :nq].reshape(q.shape), y[:, :, nq:nq + nk].reshape(k.shape),
+            y[:, :, nq + nk:].reshape(v.shape), h_out, bad)

@@ -1,6 +1,6 @@
 """Plant plausible mistakes in copies of the oracle's C source and check that the pins in
-test_oracle.py catch every one (a dropped term, a wrong sign or index, a transposed operand,
-an off-by-one commit). Mistakes are planted only in the oracle, on the CPU."""
+test_oracle.py and test_oracle_conv.py catch every one (a dropped term, a wrong sign or index,
+a transposed operand, an off-by-one commit, reversed filter taps, a history not rewound). Mistakes are planted only in the oracle, on the CPU."""
 import os
 import subprocess
 import sys
@@ -34,6 +34,13 @@ MUTANTS = {
                                   "for (int s = 0; s < t; ++s) {\n                        double d = 0.0;"),
     "chunk_handoff_decay_dropped": ("double acc = eglast * S[(int64_t)i * dk + j];",
                                     "double acc = S[(int64_t)i * dk + j];"),
+    "conv_taps_reversed": ("z += w[(int64_t)c * K + i] * xc[t + i];",
+                           "z += w[(int64_t)c * K + (K - 1 - i)] * xc[t + i];"),
+    "conv_silu_dropped": ("* C + c] = z / (1.0 + exp(-z));", "* C + c] = z;"),
+    "conv_history_not_rewound": ("const int from = ok ? L : 0;", "const int from = ok ? T : 0;"),
+    "conv_history_transposed": ("for (int r = 0; r < H; ++r) xc[r] = hist[((int64_t)b * H + r) * C + c];",
+                                "for (int r = 0; r < H; ++r) xc[r] = hist[(int64_t)b * H * C + (int64_t)c * H + r];"),
+    "conv_bad_count_commits": ("const int from = ok ? L : 0;", "const int from = ok ? L : T;"),
 }
 
 
@@ -50,6 +57,7 @@ def test_pins_catch_mutant(name, tmp_path):
                     str(c), "-lm"], check=True)
     env = dict(os.environ, GDN_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                        os.path.join(ROOT, "tests", "test_oracle.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_conv.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, r.stdout[-2000:])

@@ -421,6 +421,76 @@ const char* gdn_status_string(gdn_status status) {
 
 const char* gdn_last_error(void) { return g_last_error; }
 
+gdn_status gdn_short_conv(const gdn_shape* shape, int32_t conv_k, const void* q, const void* k,
+                          const void* v, const float* conv_w, const void* hist_in, void* hist_out,
+                          const int32_t* accept_len, void* q_out, void* k_out, void* v_out, void* stream) {
+    const char* who = "gdn_short_conv";
+    gdn_status st = check_shape(shape, 1 << 20, who);
+    if (st != GDN_OK) return st;
+    if (conv_k < 2 || conv_k > 4) return fail(GDN_ERR_UNSUPPORTED, "%s: conv_k %d not built (2, 3, 4)", who, conv_k);
+    if (shape->d_k % 8 != 0 || shape->d_v % 8 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: d_k and d_v must be multiples of 8", who);
+    const bool outputs = q_out || k_out || v_out;
+    if (outputs && !(q_out && k_out && v_out))
+        return fail(GDN_ERR_INVALID_ARG, "%s: q_out, k_out, v_out must be all given or all NULL", who);
+    if (!outputs && !hist_out) return fail(GDN_ERR_INVALID_ARG, "%s: nothing to write", who);
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(q, who);
+    REQUIRE_PTR(k, who);
+    REQUIRE_PTR(v, who);
+    REQUIRE_PTR(hist_in, who);
+    if (outputs) {
+        REQUIRE_PTR(conv_w, who);
+        REQUIRE_PTR(q_out, who);
+        REQUIRE_PTR(k_out, who);
+        REQUIRE_PTR(v_out, who);
+    }
+    if (hist_out) REQUIRE_PTR(hist_out, who);
+    if (accept_len && (reinterpret_cast<uintptr_t>(accept_len) & 3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: accept_len misaligned", who);
+    const size_t el = shape->in_dtype == GDN_BF16 ? 2 : 4;
+    const size_t qk = (size_t)shape->B * shape->T * shape->H_k * shape->d_k * el;
+    const size_t vb = (size_t)shape->B * shape->T * shape->H_v * shape->d_v * el;
+    const int64_t C = 2 * (int64_t)shape->H_k * shape->d_k + (int64_t)shape->H_v * shape->d_v;
+    const size_t hb = (size_t)shape->B * (conv_k - 1) * C * el;
+    if (hist_out && hist_out != hist_in && !overlap_ok(hist_out, hist_in, hb))
+        return fail(GDN_ERR_INVALID_ARG, "%s: hist_out partially overlaps hist_in", who);
+    if (outputs) {
+        // every output region against every input region and the history
+        const void* outs[3] = {q_out, k_out, v_out};
+        const size_t osz[3] = {qk, qk, vb};
+        const void* ins[5] = {q, k, v, hist_in, hist_out};
+        const size_t isz[5] = {qk, qk, vb, hb, hb};
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 5; ++j) {
+                if (!ins[j]) continue;
+                const char* a = static_cast<const char*>(outs[i]);
+                const char* b = static_cast<const char*>(ins[j]);
+                if (a < b + isz[j] && b < a + osz[i])
+                    return fail(GDN_ERR_INVALID_ARG, "%s: an output overlaps an input or the history", who);
+            }
+    }
+    gdn::ConvArgs c;
+    memset(&c, 0, sizeof(c));
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.w = conv_w;
+    c.hist_in = hist_in;
+    c.hist_out = hist_out;
+    c.accept_len = accept_len;
+    c.q_out = outputs ? q_out : nullptr;
+    c.k_out = outputs ? k_out : nullptr;
+    c.v_out = outputs ? v_out : nullptr;
+    c.status_word = shape->status_word;
+    c.B = shape->B;
+    c.T = shape->T;
+    c.C = (int)C;
+    c.Cq = shape->H_k * shape->d_k;
+    return launched(gdn::launch_short_conv(c, conv_k, shape->in_dtype == GDN_BF16, static_cast<cudaStream_t>(stream)),
+                    who);
+}
+
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
 
 }  // extern "C"

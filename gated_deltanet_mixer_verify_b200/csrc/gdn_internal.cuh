@@ -54,8 +54,27 @@ __host__ __device__ inline size_t stash_floats_per_head(int T, int dk, int dv) {
     return (size_t)T * dk + (((size_t)T + 3) & ~size_t(3)) + (((size_t)T * dv + 3) & ~size_t(3));
 }
 
+// Causal short convolution over q | k | v with its rewound history (gdn_conv.cu).
+struct ConvArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* w;              // [C][K] fp32
+    const void* hist_in;         // [B][K-1][C] in_dtype
+    void* hist_out;              // [B][K-1][C] in_dtype, or nullptr (history not written)
+    const int32_t* accept_len;   // [B] device, or nullptr (all T accepted)
+    void* q_out;                 // post-convolution q, k, v (in_dtype), or all nullptr
+    void* k_out;
+    void* v_out;
+    int32_t* status_word;
+    int B, T, C, Cq;             // C = 2 Cq + H_v d_v channels, Cq = H_k d_k
+    int tile;                    // tokens per thread (set by the launcher)
+    bool fused_hist;             // this launch also rewinds the history (set by the launcher)
+};
+
 // Host launchers; return cudaSuccess or the launch error. Shapes are validated by the caller.
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
+cudaError_t launch_short_conv(const ConvArgs& a, int K, bool bf16, cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);

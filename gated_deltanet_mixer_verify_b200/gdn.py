@@ -64,8 +64,10 @@ def _load():
     lib.gdn_chunk_prefill_noalloc.argtypes = [S, ctypes.c_int32] + [_VP] * 11
     lib.gdn_chunk_prefill_prepare.argtypes = [S, ctypes.c_int32] + [_VP] * 7 + [ctypes.c_size_t, _VP]
     lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
+    lib.gdn_short_conv.argtypes = [S, ctypes.c_int32] + [_VP] * 11
     for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_commit_and_verify", "gdn_chunk_prefill",
-               "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan"):
+               "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan",
+               "gdn_short_conv"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -188,6 +190,33 @@ def commit_and_verify(q, k, v, a, b, A_log, dt_bias, state, prev_stash, prev_acc
                                          _ptr(prev_accept_len), _ptr(accept_len), _ptr(o), _ptr(stash),
                                          _stream(stream)))
     return o
+
+
+def conv_channels(H_k, H_v, d_k, d_v) -> int:
+    """Channels of the short convolution: q | k | v."""
+    return 2 * H_k * d_k + H_v * d_v
+
+
+def short_conv(q, k, v, conv_w, hist_in, hist_out=None, accept_len=None, outputs=True,
+               q_out=None, k_out=None, v_out=None, status_word=None, stream=None):
+    """Causal short convolution of q, k, v (channels q | k | v, conv_w [C, K] fp32, SiLU) with
+    the history hist_in [B, K-1, C] (dtype of q), rewound into hist_out at accept_len (device
+    int32 [B]; None: all T accepted). hist_out may be hist_in (in place) or None (not written).
+    outputs=False only rewinds the history. Returns (q', k', v') or None."""
+    sh = _shape_from(q, k, v, status_word, 1e-6, 1.0, torch.float32)
+    if hist_in.dtype != q.dtype or (hist_out is not None and hist_out.dtype != q.dtype):
+        raise TypeError("the history has the dtype of q, k, v")
+    if outputs:
+        q_out = torch.empty_like(q) if q_out is None else q_out
+        k_out = torch.empty_like(k) if k_out is None else k_out
+        v_out = torch.empty_like(v) if v_out is None else v_out
+    else:
+        q_out = k_out = v_out = None
+    _check(_load().gdn_short_conv(ctypes.byref(sh), int(conv_w.shape[1]) if conv_w is not None else
+                                  int(hist_in.shape[1]) + 1, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                  _ptr(hist_in), _ptr(hist_out), _ptr(accept_len), _ptr(q_out), _ptr(k_out),
+                                  _ptr(v_out), _stream(stream)))
+    return (q_out, k_out, v_out) if outputs else None
 
 
 def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale=1.0,

@@ -128,6 +128,19 @@ def make_inputs(w: Workload, layer: int = 0, gates: str = "config",
     }
 
 
+def make_conv_inputs(w: Workload, K: int = 4, layer: int = 0) -> dict:
+    """Synthetic short-convolution parameters for workload ``w`` (CPU torch tensors):
+    conv_w [C, K] fp32 ~ U(-1/sqrt(K), 1/sqrt(K)) (a depthwise filter's default init) and
+    hist [B, K-1, C] ~ N(0, 1) in the workload's input dtype, C = 2 H_k d_k + H_v d_v
+    (channels q | k | v). Its own stream, (seed, layer, 7), so the mixer inputs are unchanged."""
+    rng = np.random.default_rng([w.seed, layer, 7])
+    C = 2 * w.H_k * w.d_k + w.H_v * w.d_v
+    bound = 1.0 / np.sqrt(K)
+    conv_w = rng.uniform(-bound, bound, size=(C, K)).astype(np.float32)
+    hist = rng.standard_normal((w.B, K - 1, C), dtype=np.float32)
+    return {"conv_w": torch.from_numpy(conv_w), "hist": _store(hist, w.in_dtype)}
+
+
 def as_f64(inputs: dict) -> dict:
     """The same inputs as float64 NumPy arrays (exact: every stored value is representable)."""
     out = {}

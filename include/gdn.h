@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 3   /* 3: gdn_commit_and_verify; 2: prefill split into prepare / scan */
+#define GDN_ABI_VERSION 4   /* 4: gdn_short_conv; 3: gdn_commit_and_verify; 2: prefill split into prepare / scan */
 
 typedef enum {
     GDN_OK = 0,
@@ -246,6 +246,39 @@ gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk,
                                      const float* A_log, const float* dt_bias,
                                      const float* state_in, float* state_out, void* o,
                                      void* stream);
+
+/*
+ * gdn_short_conv -- the causal short convolution in front of the mixer (one filter of conv_k
+ * taps per channel, SiLU after the sum, no bias) with the filter's short history, rewound to
+ * the accepted prefix. That history is one of the three structures brought back in line with
+ * the accepted tokens after a verify block ("Qwen 3.8 27B mac m5: 200 tok/s, audited",
+ * section "How does DSpark speculative decoding create more than one token per read?"); the
+ * page fixes no width or activation, and this is the plain reading of it.
+ * Channels are ordered q | k | v: C = 2 H_k d_k + H_v d_v; channel g d_k + j is q head g,
+ * column j; H_k d_k + g d_k + j is k; 2 H_k d_k + h d_v + j is v. Per sequence b, channel c:
+ *   xc = [hist_in rows 0 .. conv_k - 2 (oldest first), the block's inputs x_0 .. x_{T-1}]
+ *   out_t = silu(sum_{i < conv_k} conv_w[c][i] xc[t + i])   (conv_w[c][conv_k - 1] weighs x_t)
+ *   hist_out rows = xc[L .. L + conv_k - 2],  L = accept_len[b] (L = T when accept_len is NULL)
+ *   shape          B, T, H_k, H_v, d_k, d_v, in_dtype (inputs, outputs and history alike) and
+ *                  status_word; d_k and d_v multiples of 8; T up to 2^20.
+ *   conv_k         filter taps: 2, 3 or 4 (else GDN_ERR_UNSUPPORTED).
+ *   q, k, v        the block's inputs before the convolution, layouts as gdn_verify_step.
+ *   conv_w         [C][conv_k] fp32.
+ *   hist_in        [B][conv_k - 1][C] in_dtype: the last conv_k - 1 inputs before the block.
+ *   hist_out       same layout, or NULL (history not written: two-phase, rewind later by a
+ *                  call with NULL outputs). May equal hist_in (rewound in place).
+ *   accept_len     [B] int32, device, or NULL. An out-of-range count keeps the old history
+ *                  and sets status bit 1 (GDN_STATUS_BAD_ACCEPT).
+ *   q_out, k_out, v_out  the convolved q, k, v (layouts of q, k, v), all given or all NULL
+ *                  (history rewind only). They must not overlap the inputs or the history.
+ * Everything is caller-owned device memory, 16-byte aligned. The arithmetic is fp32; outputs
+ * are rounded once to in_dtype. History rows are copies of inputs, so a rewind is exact.
+ * Returns GDN_ERR_INVALID_ARG when q_out, k_out, v_out and hist_out are all NULL.
+ */
+gdn_status gdn_short_conv(const gdn_shape* shape, int32_t conv_k,
+                          const void* q, const void* k, const void* v, const float* conv_w,
+                          const void* hist_in, void* hist_out, const int32_t* accept_len,
+                          void* q_out, void* k_out, void* v_out, void* stream);
 
 /* Bytes of stash gdn_verify_step writes for this shape (0 for an invalid shape). */
 size_t gdn_stash_bytes(const gdn_shape* shape);

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 3
+    assert lib.gdn_abi_version() == 4
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -141,3 +141,31 @@ def test_commit_and_verify_validates_on_the_host(gdn):
     assert call(8, shape=gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=96, d_v=128)) == UNSUP
     empty = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
     assert lib.gdn_commit_and_verify(ctypes.byref(empty), 8, *([None] * 13), None) == 0
+
+
+def test_short_conv_validates_on_the_host(gdn):
+    INVALID, UNSUP = -1, -2
+    lib = gdn.lib()
+    fake = 0x100000
+    sh = gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    C = gdn.conv_channels(16, 48, 128, 128)
+    assert C == 10240
+    hist_bytes = 2 * 3 * C * 2
+    call = lambda K=4, **kw: lib.gdn_short_conv(
+        ctypes.byref(kw.get("shape", sh)), K, kw.get("q", fake), fake, fake, kw.get("w", fake), kw.get("h", fake),
+        kw.get("ho", fake), None, kw.get("qo", 0x4000000), kw.get("ko", 0x5000000), kw.get("vo", 0x6000000), None)
+    assert call(K=5) == UNSUP and "conv_k" in lib.gdn_last_error().decode()
+    assert call(K=1) == UNSUP
+    assert call(shape=gdn.make_shape(B=2, T=8, H_k=1, H_v=1, d_k=16, d_v=12)) == UNSUP
+    assert call(ko=None) == INVALID and "all given or all NULL" in lib.gdn_last_error().decode()
+    assert call(qo=None, ko=None, vo=None, ho=None) == INVALID and "nothing to write" in lib.gdn_last_error().decode()
+    assert call(q=None) == INVALID and "q is NULL" in lib.gdn_last_error().decode()
+    assert call(w=None) == INVALID and "conv_w is NULL" in lib.gdn_last_error().decode()
+    assert call(h=fake + 8) == INVALID and "not 16-byte aligned" in lib.gdn_last_error().decode()
+    assert call(ho=fake + 16) == INVALID and "partially overlaps" in lib.gdn_last_error().decode()
+    assert call(qo=fake) == INVALID and "overlaps" in lib.gdn_last_error().decode()       # output on an input
+    assert call(vo=fake + hist_bytes - 16, h=fake + 0x2000000, ho=fake + hist_bytes - 32 + 0x2000000) == INVALID
+    # rewind only: no weights needed
+    empty = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    assert lib.gdn_short_conv(ctypes.byref(empty), 4, *([None] * 6), None, None, None, None, None) == INVALID
+    assert lib.gdn_short_conv(ctypes.byref(empty), 4, *([None] * 5), fake, None, None, None, None, None) == 0

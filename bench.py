@@ -45,7 +45,9 @@ KERNEL_SOURCES = {
     "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
+    "short_conv": [_CSRC + "gdn_conv.cu"] + _HEADERS,
 }
+CONV_K, CONV_LAYERS = 4, 48   # short convolution: filter taps; one convolution per GDN layer
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -162,8 +164,26 @@ def commit_next_bytes(w):
     return algorithmic_bytes(w, n_state_writes=w.B) + 2 * stash
 
 
+def conv_bytes(w, K=CONV_K):
+    """Bytes one short-convolution launch must move: q, k, v read and written once, the
+    history read and rewound, the taps and the accept counts."""
+    el = 2 if w.in_dtype == "bf16" else 4
+    C = 2 * w.H_k * w.d_k + w.H_v * w.d_v
+    return 2 * w.B * w.T * C * el + 2 * w.B * (K - 1) * C * el + C * K * 4 + w.B * 4
+
+
 def workload_config(name):
     """The JSON `config` of a workload (what it is, with its sizes)."""
+    if name == "short_conv":
+        c = workload_config("batched_verify")
+        w = workload("batched_verify")
+        c.update(workload=name, conv_k=CONV_K, layers=CONV_LAYERS,
+                 channels="q | k | v: %d" % (2 * w.H_k * w.d_k + w.H_v * w.d_v),
+                 accept_len="min(Geometric(0.25), 8) per sequence, device int32",
+                 state="short history [B, K-1, C] bf16 per layer, rewound in place",
+                 launch="%d launches (one per layer, distinct buffers) captured in one CUDA graph" % CONV_LAYERS,
+                 l2="inputs larger than L2 (%.0f MB moved per step, L2 126 MB)" % (conv_bytes(w) * CONV_LAYERS / 1e6))
+        return c
     if name == "commit_next_verify":
         c = workload_config("batched_verify")
         w = workload("batched_verify")
@@ -256,6 +276,80 @@ class CommitNext(Verify):
 
     def config(self):
         return workload_config("commit_next_verify")
+
+
+class ShortConv:
+    """short_conv: the causal short convolution of one verify block (B = 64, T = 8) for each of
+    48 layers, each with its own inputs, taps and history, captured once as a CUDA graph; a
+    step replays the graph."""
+
+    def __init__(self, name, rank, dev):
+        from gated_deltanet_mixer_verify_b200 import gdn
+        from gated_deltanet_mixer_verify_b200.inputs import make_conv_block
+        self.gdn = gdn
+        self.w = workload("batched_verify", seed=rank_seed(workload("batched_verify").seed, rank))
+        self.layers = []
+        for l in range(CONV_LAYERS):
+            x = make_conv_block(self.w, K=CONV_K, layer=l)
+            if l == 0:
+                self.host = x
+            xd = {k: v.to(dev) for k, v in x.items()}
+            xd.update(qo=torch.empty_like(xd["q"]), ko=torch.empty_like(xd["k"]), vo=torch.empty_like(xd["v"]))
+            self.layers.append(xd)
+        self.launches_per_step = CONV_LAYERS
+        self.bytes = conv_bytes(self.w) * CONV_LAYERS
+        self.units = self.w.B * self.w.T * self.w.H_v * CONV_LAYERS
+        self.graph = None
+        self.stream = torch.cuda.Stream(dev)
+
+    def conv(self, x):
+        self.gdn.short_conv(x["q"], x["k"], x["v"], x["conv_w"], x["hist"], x["hist"], x["accept_len"],
+                            q_out=x["qo"], k_out=x["ko"], v_out=x["vo"], stream=self.stream)
+
+    def step(self):
+        if self.graph is None:
+            with torch.cuda.stream(self.stream):
+                for x in self.layers:
+                    self.conv(x)                                  # warm the launch path
+            torch.cuda.current_stream().wait_stream(self.stream)
+            torch.cuda.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                for x in self.layers:
+                    self.conv(x)
+        self.graph.replay()
+
+    def e2e(self, steps, barrier, world, dev):
+        """Through the public call with host buffers: per step, one layer's q, k, v and accept
+        counts copied in from pinned memory, the convolution, its q', k', v' copied out."""
+        names = ["q", "k", "v", "accept_len"]
+        host = {k: self.host[k].pin_memory() for k in names}
+        x = dict(self.layers[0])
+        x.update({k: torch.empty_like(self.layers[0][k]) for k in names})
+        outs = [torch.empty(x[k].shape, dtype=x[k].dtype).pin_memory() for k in ("qo", "ko", "vo")]
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(steps):
+            for k in names:
+                x[k].copy_(host[k], non_blocking=True)
+            self.gdn.short_conv(x["q"], x["k"], x["v"], x["conv_w"], x["hist"], x["hist"], x["accept_len"],
+                                q_out=x["qo"], k_out=x["ko"], v_out=x["vo"])
+            for o, k in zip(outs, ("qo", "ko", "vo")):
+                o.copy_(x[k], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_s = max_over_ranks(e0.elapsed_time(e1)) / steps / 1e3
+        h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        return {"value": weak_scaling_throughput(conv_bytes(self.w), world, e_s) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    def config(self):
+        return workload_config("short_conv")
 
 
 class SingleSeq:
@@ -351,7 +445,7 @@ class Prefill:
 
 
 WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
-             "prefill": Prefill, "commit_next_verify": CommitNext}
+             "prefill": Prefill, "commit_next_verify": CommitNext, "short_conv": ShortConv}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -361,9 +455,27 @@ def oracle_sample(name, budget_s, rank=0):
     Returns (seconds per unit, units timed, description, threads)."""
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    shape = "batched_verify" if name == "commit_next_verify" else name
+    shape = "batched_verify" if name in ("commit_next_verify", "short_conv") else name
     w = workload(shape, seed=rank_seed(workload(shape).seed, rank))
     threads = orc.max_threads()
+    if name == "short_conv":
+        from gated_deltanet_mixer_verify_b200.inputs import make_conv_block
+        n_seq = 16
+        sub = workload(shape, B=n_seq)
+        blk = make_conv_block(sub, K=CONV_K)
+        f = {k: v.double().numpy() for k, v in blk.items() if k != "accept_len"}
+        L = blk["accept_len"].numpy()
+        reps, t_total = 0, 0.0
+        while t_total < budget_s or reps == 0:
+            t0 = time.perf_counter()
+            orc.short_conv(f["q"], f["k"], f["v"], f["conv_w"], f["hist"], L)
+            t_total += time.perf_counter() - t0
+            reps += 1
+            if reps >= 1000:
+                break
+        desc = "%d sequences x %d channels x T=%d, K=%d, %d repetition(s)" % (
+            n_seq, 2 * w.H_k * w.d_k + w.H_v * w.d_v, w.T, CONV_K, reps)
+        return t_total / (reps * n_seq), n_seq * reps, desc, 1
     if name == "prefill":
         sub = workload(name, T=2048, H_k=1, H_v=3)
         f = as_f64(make_inputs(sub))
@@ -396,7 +508,9 @@ def cpu_value(name, per_unit_s):
     """The workload metric (GB/s or tok/s) the oracle reaches at per_unit_s per unit."""
     if name == "prefill":
         return 1.0 / per_unit_s, "tok/s"
-    if name == "commit_next_verify":
+    if name == "short_conv":
+        per_seq_bytes = conv_bytes(workload("batched_verify", B=1))
+    elif name == "commit_next_verify":
         per_seq_bytes = commit_next_bytes(workload("batched_verify", B=1))
     else:
         per_seq_bytes = algorithmic_bytes(workload(name, B=1))
@@ -421,6 +535,15 @@ def run_reference(args, rank, world):
                                   f["dt_bias"], None)
         units_per_step = 256 * 3 / workload(name).H_v          # prompt tokens (all heads)
         desc = "256 tokens x 3 of 48 value heads per step (fp64 recurrence)"
+    elif name == "short_conv":
+        from gated_deltanet_mixer_verify_b200.inputs import make_conv_block
+        sub = workload("batched_verify", B=4)
+        blk = make_conv_block(sub, K=CONV_K)
+        f = {k: v.double().numpy() for k, v in blk.items() if k != "accept_len"}
+        L = blk["accept_len"].numpy()
+        run = lambda: orc.short_conv(f["q"], f["k"], f["v"], f["conv_w"], f["hist"], L)
+        units_per_step = conv_bytes(sub) / 1e9
+        desc = "4 sequences x 10240 channels x T=8, K=%d per step (one layer)" % CONV_K
     else:
         n_seq = 16 if name == "decode" else 1
         shape = "batched_verify" if name == "commit_next_verify" else name
@@ -446,7 +569,8 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference", "config": workload_config(name),
-            "cpu_baseline": {"value": value, "unit": unit, "cores": orc.max_threads(),
+            "cpu_baseline": {"value": value, "unit": unit,
+                             "cores": 1 if name == "short_conv" else orc.max_threads(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -523,7 +647,9 @@ def main():
 
     # end to end through the public API: pinned host inputs -> device -> mixer -> host output
     e2e = None
-    if isinstance(wl, (Verify, Prefill)):
+    if hasattr(wl, "e2e"):
+        e2e = wl.e2e(args.steps, barrier, world, dev)
+    elif isinstance(wl, (Verify, Prefill)):
         names = wl.per_step_inputs()
         host = {k: wl.host[k].pin_memory() for k in names}
         dev_in = dict(wl.x)
@@ -605,7 +731,7 @@ def main():
                                     "sample": desc}
         print(json.dumps(line), flush=True)
 
-    if isinstance(wl, SingleSeq):
+    if isinstance(wl, (SingleSeq, ShortConv)):
         wl.graph = None
     if world > 1:
         barrier()

@@ -141,6 +141,24 @@ def make_conv_inputs(w: Workload, K: int = 4, layer: int = 0) -> dict:
     return {"conv_w": torch.from_numpy(conv_w), "hist": _store(hist, w.in_dtype)}
 
 
+def make_conv_block(w: Workload, K: int = 4, layer: int = 0) -> dict:
+    """One layer's inputs of the short convolution alone (no recurrent state): q, k, v
+    ~ N(0, 1) before the convolution (the workload's layouts and input dtype), accept_len as
+    the workload draws it, and conv_w, hist as :func:`make_conv_inputs`. Its own stream,
+    (seed, layer, 8)."""
+    rng = np.random.default_rng([w.seed, layer, 8])
+    B, T, Hk, Hv, dk, dv = w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v
+    f32 = np.float32
+    q = rng.standard_normal((B, T, Hk, dk), dtype=f32)
+    k = rng.standard_normal((B, T, Hk, dk), dtype=f32)
+    v = rng.standard_normal((B, T, Hv, dv), dtype=f32)
+    L = np.minimum(rng.geometric(0.25, size=B), T).astype(np.int32)
+    out = {"q": _store(q, w.in_dtype), "k": _store(k, w.in_dtype), "v": _store(v, w.in_dtype),
+           "accept_len": torch.from_numpy(L)}
+    out.update(make_conv_inputs(w, K=K, layer=layer))
+    return out
+
+
 def as_f64(inputs: dict) -> dict:
     """The same inputs as float64 NumPy arrays (exact: every stored value is representable)."""
     out = {}

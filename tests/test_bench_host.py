@@ -50,3 +50,19 @@ def test_reference_arm_commit_next_verify():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["config"]["workload"] == "commit_next_verify"
     assert d["unit"] == "GB/s" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_conv_bytes(bench):
+    w = workload("batched_verify")
+    C = 2 * 16 * 128 + 48 * 128
+    # q, k, v in and out (bf16), history in and out (3 rows), taps (fp32), accept counts
+    assert bench.conv_bytes(w) == 2 * 64 * 8 * C * 2 + 2 * 64 * 3 * C * 2 + C * 4 * 4 + 64 * 4
+
+
+def test_reference_arm_short_conv():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "short_conv", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"]["workload"] == "short_conv" and d["cpu_baseline"]["cores"] == 1 and d["value"] > 0

@@ -76,3 +76,20 @@ def test_bf16_rounding_is_round_to_nearest_even():
     # every stored value is a bf16 value: its float32 bit pattern has 16 zero low bits
     bits = x["q"].float().view(torch.int32)
     assert int((bits & 0xFFFF).abs().max()) == 0
+
+
+def test_conv_inputs_shapes_ranges_and_streams():
+    from gated_deltanet_mixer_verify_b200.inputs import make_conv_block, make_conv_inputs
+    w = workload("batched_verify", B=3)
+    C = 2 * w.H_k * w.d_k + w.H_v * w.d_v
+    c = make_conv_inputs(w, K=4)
+    assert c["conv_w"].shape == (C, 4) and c["conv_w"].dtype == torch.float32
+    assert float(c["conv_w"].abs().max()) <= 0.5                     # U(-1/sqrt(K), 1/sqrt(K))
+    assert c["hist"].shape == (3, 3, C) and c["hist"].dtype == torch.bfloat16
+    blk = make_conv_block(w, K=3, layer=2)
+    assert blk["q"].shape == (3, 8, 16, 128) and blk["v"].shape == (3, 8, 48, 128)
+    assert blk["hist"].shape == (3, 2, C)
+    assert 1 <= int(blk["accept_len"].min()) and int(blk["accept_len"].max()) <= 8
+    # the mixer's own inputs are untouched by the convolution streams
+    assert torch.equal(make_inputs(w)["q"], make_inputs(w)["q"])
+    assert not torch.equal(make_conv_block(w, layer=2)["q"], make_conv_block(w, layer=3)["q"])

@@ -353,3 +353,26 @@ int oracle_short_conv(int B, int T, int C, int K, const double* x, const double*
     free(xc);
     return bad;
 }
+
+/*
+ * Gated RMS normalisation of the mixer's output. The source ("Lithos-metal: Qwen3.8-27B on
+ * 40-core M5 Max", table "GDN mixer") lists gating and normalisation among the mixer's jobs,
+ * after the recurrence, without the formula; this is the plain reading, per output row
+ * (one token of one value head, d values):
+ *   y_j = o_j / sqrt( (1/d) sum_j o_j^2 + eps ) * w_j * silu(z_j),   silu(z) = z / (1 + e^-z)
+ * o, z, y: [n][d]; w: [d] (shared by all rows).
+ */
+void oracle_gated_rmsnorm(int64_t n, int d, const double* o, const double* z, const double* w, double eps,
+                          double* y) {
+    for (int64_t r = 0; r < n; ++r) {
+        const double* orow = o + r * d;
+        const double* zrow = z + r * d;
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) ss += orow[j] * orow[j];
+        const double inv = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j) {
+            const double g = zrow[j] / (1.0 + exp(-zrow[j]));
+            y[r * d + j] = orow[j] * inv * w[j] * g;
+        }
+    }
+}

@@ -46,6 +46,8 @@ def _load():
         lib.oracle_chunked.restype = ctypes.c_int
         lib.oracle_short_conv.argtypes = [ctypes.c_int] * 4 + [_D] * 3 + [_I32, _D, _D]
         lib.oracle_short_conv.restype = ctypes.c_int
+        lib.oracle_gated_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int, _D, _D, _D, ctypes.c_double, _D]
+        lib.oracle_gated_rmsnorm.restype = None
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -200,3 +202,15 @@ def short_conv(q, k, v, w, hist, accept_len=None, write_history=True):
     nq, nk = int(np.prod(q.shape[2:])), int(np.prod(k.shape[2:]))
     return (y[:, :, :nq].reshape(q.shape), y[:, :, nq:nq + nk].reshape(k.shape),
             y[:, :, nq + nk:].reshape(v.shape), h_out, bad)
+
+
+def gated_rmsnorm(o, z, w, eps=1e-6):
+    """Gated RMS normalisation over the last axis (oracle_gated_rmsnorm):
+    y = o / sqrt(mean(o^2) + eps) * w * silu(z). o, z: [..., d]; w: [d]."""
+    o, z, w = _f64(o), _f64(z), _f64(w)
+    d = o.shape[-1]
+    if z.shape != o.shape or w.shape != (d,):
+        raise ValueError("gated_rmsnorm: inconsistent shape")
+    y = np.empty_like(o)
+    _load().oracle_gated_rmsnorm(o.size // d if d else 0, d, _p(o), _p(z), _p(w), float(eps), _p(y))
+    return y

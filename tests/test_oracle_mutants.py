@@ -1,5 +1,5 @@
 """Plant plausible mistakes in copies of the oracle's C source and check that the pins in
-test_oracle.py and test_oracle_conv.py catch every one (a dropped term, a wrong sign or index,
+test_oracle.py, test_oracle_conv.py and test_oracle_norm.py catch every one (a dropped term, a wrong sign or index,
 a transposed operand, an off-by-one commit, reversed filter taps, a history not rewound). Mistakes are planted only in the oracle, on the CPU."""
 import os
 import subprocess
@@ -41,6 +41,12 @@ MUTANTS = {
     "conv_history_transposed": ("for (int r = 0; r < H; ++r) xc[r] = hist[((int64_t)b * H + r) * C + c];",
                                 "for (int r = 0; r < H; ++r) xc[r] = hist[(int64_t)b * H * C + (int64_t)c * H + r];"),
     "conv_bad_count_commits": ("const int from = ok ? L : 0;", "const int from = ok ? L : T;"),
+    "norm_sum_not_mean": ("1.0 / sqrt(ss / d + eps);", "1.0 / sqrt(ss + eps);"),
+    "norm_eps_outside_sqrt": ("1.0 / sqrt(ss / d + eps);", "1.0 / (sqrt(ss / d) + eps);"),
+    "norm_gate_sigmoid_not_silu": ("const double g = zrow[j] / (1.0 + exp(-zrow[j]));",
+                                   "const double g = 1.0 / (1.0 + exp(-zrow[j]));"),
+    "norm_weight_dropped": ("y[r * d + j] = orow[j] * inv * w[j] * g;", "y[r * d + j] = orow[j] * inv * g;"),
+    "norm_gate_on_wrong_row": ("const double* zrow = z + r * d;", "const double* zrow = z;"),
 }
 
 
@@ -58,6 +64,7 @@ def test_pins_catch_mutant(name, tmp_path):
     env = dict(os.environ, GDN_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_conv.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_conv.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_norm.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, r.stdout[-2000:])

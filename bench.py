@@ -42,6 +42,7 @@ _HEADERS = [_CSRC + f for f in ("gdn_tc.cuh", "gdn_device.cuh", "gdn_internal.cu
 KERNEL_SOURCES = {
     "batched_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "commit_next_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
+    "verify_gated": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
@@ -172,8 +173,22 @@ def conv_bytes(w, K=CONV_K):
     return 2 * w.B * w.T * C * el + 2 * w.B * (K - 1) * C * el + C * K * 4 + w.B * 4
 
 
+def gated_bytes(w):
+    """Bytes of a verify call with the gated output normalisation: the verify call's, plus the
+    gate z (v's size) and the d_v weights."""
+    el = 2 if w.in_dtype == "bf16" else 4
+    return algorithmic_bytes(w) + w.B * w.T * w.H_v * w.d_v * el + w.d_v * 4
+
+
 def workload_config(name):
     """The JSON `config` of a workload (what it is, with its sizes)."""
+    if name == "verify_gated":
+        c = workload_config("batched_verify")
+        w = workload("batched_verify")
+        c.update(workload=name, norm="o / sqrt(mean(o^2) + 1e-6) * w * silu(z) per (token, value head), "
+                 "z bf16 like v, w fp32 [d_v]; fused into the verify kernel's outputs",
+                 l2="inputs larger than L2 (%.0f MB moved per step, L2 126 MB)" % (gated_bytes(w) / 1e6))
+        return c
     if name == "short_conv":
         c = workload_config("batched_verify")
         w = workload("batched_verify")
@@ -247,6 +262,31 @@ class Verify:
 
     def per_step_inputs(self):
         return ["q", "k", "v", "a", "b"] + ([] if self.decode else ["accept_len"])
+
+
+class VerifyGated(Verify):
+    """verify_gated: batched verify whose outputs carry the gated RMS normalisation (one call,
+    the normalisation applied by the verify kernel to its outputs)."""
+
+    def __init__(self, name, rank, dev):
+        super().__init__("batched_verify", rank, dev)
+        from gated_deltanet_mixer_verify_b200.inputs import make_norm_inputs
+        n = make_norm_inputs(self.w)
+        self.host.update(n)
+        self.x.update({k: v.to(dev) for k, v in n.items()})
+        self.bytes = gated_bytes(self.w)
+
+    def step(self, x=None, o=None):
+        x = x or self.x
+        o = self.o if o is None else o
+        self.gdn.verify_step_gated(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"], self.state,
+                                   self.state, x["accept_len"], x["norm_z"], x["norm_w"], 1e-6, o=o)
+
+    def per_step_inputs(self):
+        return super().per_step_inputs() + ["norm_z"]
+
+    def config(self):
+        return workload_config("verify_gated")
 
 
 class CommitNext(Verify):
@@ -445,7 +485,8 @@ class Prefill:
 
 
 WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
-             "prefill": Prefill, "commit_next_verify": CommitNext, "short_conv": ShortConv}
+             "prefill": Prefill, "commit_next_verify": CommitNext, "short_conv": ShortConv,
+             "verify_gated": VerifyGated}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -455,7 +496,7 @@ def oracle_sample(name, budget_s, rank=0):
     Returns (seconds per unit, units timed, description, threads)."""
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    shape = "batched_verify" if name in ("commit_next_verify", "short_conv") else name
+    shape = "batched_verify" if name in ("commit_next_verify", "short_conv", "verify_gated") else name
     w = workload(shape, seed=rank_seed(workload(shape).seed, rank))
     threads = orc.max_threads()
     if name == "short_conv":
@@ -485,14 +526,20 @@ def oracle_sample(name, budget_s, rank=0):
         # units are tokens of all 48 heads: 3 of 48 heads timed over 2048 tokens
         per_token = dt / 2048 * (w.H_v / 3)
         return per_token, 2048, "2048 tokens x 3 of 48 value heads (fp64 recurrence)", threads
-    n_seq = {"batched_verify": 8, "decode": 64, "single_seq_verify": 1, "commit_next_verify": 8}[name]
+    n_seq = {"batched_verify": 8, "decode": 64, "single_seq_verify": 1, "commit_next_verify": 8,
+             "verify_gated": 8}[name]
     sub = workload(shape, B=n_seq)
     f = as_f64(make_inputs(sub))
     L = f["accept_len"] if name != "decode" else None
+    if name == "verify_gated":
+        from gated_deltanet_mixer_verify_b200.inputs import make_norm_inputs
+        nrm = {k: v.double().numpy() for k, v in make_norm_inputs(sub).items()}
     reps, t_total = 0, 0.0
     while t_total < budget_s or reps == 0:
         t0 = time.perf_counter()
-        orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"], f["S0"], L)
+        o, _, _ = orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"], f["dt_bias"], f["S0"], L)
+        if name == "verify_gated":
+            orc.gated_rmsnorm(o, nrm["norm_z"], nrm["norm_w"], 1e-6)
         t_total += time.perf_counter() - t0
         reps += 1
         if reps >= 1000:
@@ -510,6 +557,8 @@ def cpu_value(name, per_unit_s):
         return 1.0 / per_unit_s, "tok/s"
     if name == "short_conv":
         per_seq_bytes = conv_bytes(workload("batched_verify", B=1))
+    elif name == "verify_gated":
+        per_seq_bytes = gated_bytes(workload("batched_verify", B=1))
     elif name == "commit_next_verify":
         per_seq_bytes = commit_next_bytes(workload("batched_verify", B=1))
     else:
@@ -546,13 +595,21 @@ def run_reference(args, rank, world):
         desc = "4 sequences x 10240 channels x T=8, K=%d per step (one layer)" % CONV_K
     else:
         n_seq = 16 if name == "decode" else 1
-        shape = "batched_verify" if name == "commit_next_verify" else name
+        shape = "batched_verify" if name in ("commit_next_verify", "verify_gated") else name
         sub = workload(shape, B=n_seq)
         f = as_f64(make_inputs(sub))
         L = None if name == "decode" else f["accept_len"]
-        run = lambda: orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
-                                 f["dt_bias"], f["S0"], L)
-        per_step = commit_next_bytes(sub) if name == "commit_next_verify" else algorithmic_bytes(sub)
+        if name == "verify_gated":
+            from gated_deltanet_mixer_verify_b200.inputs import make_norm_inputs
+            nrm = {k: v.double().numpy() for k, v in make_norm_inputs(sub).items()}
+            run = lambda: orc.gated_rmsnorm(orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
+                                                       f["dt_bias"], f["S0"], L)[0],
+                                            nrm["norm_z"], nrm["norm_w"], 1e-6)
+        else:
+            run = lambda: orc.verify(f["q"], f["k"], f["v"], f["a"], f["b"], f["A_log"],
+                                     f["dt_bias"], f["S0"], L)
+        per_step = {"commit_next_verify": commit_next_bytes, "verify_gated": gated_bytes}.get(
+            name, algorithmic_bytes)(sub)
         units_per_step = per_step / 1e9                        # GB of the workload per step
         desc = "%d sequence(s) x 48 value heads x T=%d per step" % (n_seq, sub.T)
         if name == "commit_next_verify":

@@ -106,15 +106,18 @@ gdn_status launched(cudaError_t e, const char* who) {
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-gdn_status gdn_verify_step(const gdn_shape* shape, const void* q, const void* k, const void* v,
-                           const void* a, const void* b, const float* A_log, const float* dt_bias,
-                           const float* state_in, float* state_out, const int32_t* accept_len,
-                           void* o, float* stash, void* stream) {
-    const char* who = "gdn_verify_step";
+// gdn_verify_step and gdn_verify_step_gated (norm_z non-NULL: gated norm of the outputs).
+gdn_status verify_impl(const char* who, const gdn_shape* shape, const void* q, const void* k, const void* v,
+                       const void* a, const void* b, const float* A_log, const float* dt_bias,
+                       const float* state_in, float* state_out, const int32_t* accept_len, const void* norm_z,
+                       const float* norm_w, float norm_eps, void* o, float* stash, void* stream) {
     gdn_status st = check_shape(shape, 16, who);
     if (st != GDN_OK) return st;
+    if (norm_z && shape->d_v % 4 != 0)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: the gated norm needs d_v a multiple of 4", who);
+    if (norm_z && !(norm_eps >= 0.f)) return fail(GDN_ERR_INVALID_ARG, "%s: norm_eps must be >= 0", who);
     if (shape->B == 0) return ok();
     REQUIRE_PTR(q, who);
     REQUIRE_PTR(k, who);
@@ -125,6 +128,10 @@ gdn_status gdn_verify_step(const gdn_shape* shape, const void* q, const void* k,
     REQUIRE_PTR(dt_bias, who);
     REQUIRE_PTR(state_in, who);
     REQUIRE_PTR(o, who);
+    if (norm_z) {
+        REQUIRE_PTR(norm_z, who);
+        REQUIRE_PTR(norm_w, who);
+    }
     if (accept_len) {
         REQUIRE_PTR(accept_len, who);
         REQUIRE_PTR(state_out, who);
@@ -141,7 +148,72 @@ gdn_status gdn_verify_step(const gdn_shape* shape, const void* q, const void* k,
     x.o = o;
     x.stash = stash;
     x.always_commit = 0;
+    x.norm_z = norm_z;
+    x.norm_w = norm_w;
+    x.norm_eps = norm_eps;
     return launched(gdn::launch_verify(x, static_cast<cudaStream_t>(stream)), who);
+}
+
+}  // namespace
+
+extern "C" {
+
+
+gdn_status gdn_verify_step(const gdn_shape* shape, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, const float* A_log, const float* dt_bias,
+                           const float* state_in, float* state_out, const int32_t* accept_len,
+                           void* o, float* stash, void* stream) {
+    return verify_impl("gdn_verify_step", shape, q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept_len,
+                       nullptr, nullptr, 0.f, o, stash, stream);
+}
+
+gdn_status gdn_verify_step_gated(const gdn_shape* shape, const void* q, const void* k, const void* v,
+                                 const void* a, const void* b, const float* A_log, const float* dt_bias,
+                                 const float* state_in, float* state_out, const int32_t* accept_len,
+                                 const void* norm_z, const float* norm_w, float norm_eps, void* o, float* stash,
+                                 void* stream) {
+    const char* who = "gdn_verify_step_gated";
+    if (!norm_z) return fail(GDN_ERR_INVALID_ARG, "%s: norm_z is NULL", who);
+    return verify_impl(who, shape, q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept_len, norm_z, norm_w,
+                       norm_eps, o, stash, stream);
+}
+
+gdn_status gdn_gated_rmsnorm(int64_t rows, int32_t d, const void* x, int32_t x_dtype, const void* z,
+                             int32_t z_dtype, const float* w, float eps, void* y, int32_t y_dtype, void* stream) {
+    const char* who = "gdn_gated_rmsnorm";
+    if (rows < 0 || d < 4 || d % 4 != 0 || d > 4096)
+        return fail(GDN_ERR_INVALID_ARG, "%s: rows >= 0 and d a multiple of 4 in 4..4096 required", who);
+    for (int32_t t : {x_dtype, z_dtype, y_dtype})
+        if (t != GDN_F32 && t != GDN_BF16) return fail(GDN_ERR_INVALID_ARG, "%s: dtype %d unknown", who, t);
+    if (!(eps >= 0.f)) return fail(GDN_ERR_INVALID_ARG, "%s: eps must be >= 0", who);
+    if (rows > ((int64_t)1 << 33)) return fail(GDN_ERR_UNSUPPORTED, "%s: more than 2^33 rows", who);
+    if (rows == 0) return ok();
+    REQUIRE_PTR(x, who);
+    REQUIRE_PTR(z, who);
+    REQUIRE_PTR(w, who);
+    REQUIRE_PTR(y, who);
+    const size_t xb = (size_t)rows * d * (x_dtype == GDN_BF16 ? 2 : 4);
+    const size_t yb = (size_t)rows * d * (y_dtype == GDN_BF16 ? 2 : 4);
+    if (x != y) {
+        const char* xp = static_cast<const char*>(x);
+        const char* yp = static_cast<const char*>(y);
+        if (xp < yp + yb && yp < xp + xb)
+            return fail(GDN_ERR_INVALID_ARG, "%s: y partially overlaps x", who);
+    } else if (x_dtype != y_dtype) {
+        return fail(GDN_ERR_INVALID_ARG, "%s: in place needs x and y of one dtype", who);
+    }
+    gdn::NormArgs n;
+    n.x = x;
+    n.z = z;
+    n.w = w;
+    n.y = y;
+    n.rows = rows;
+    n.d = d;
+    n.eps = eps;
+    n.x_bf16 = x_dtype == GDN_BF16;
+    n.z_bf16 = z_dtype == GDN_BF16;
+    n.y_bf16 = y_dtype == GDN_BF16;
+    return launched(gdn::launch_gated_rmsnorm(n, static_cast<cudaStream_t>(stream)), who);
 }
 
 gdn_status gdn_commit(const gdn_shape* shape, const float* state_in, float* state_out,

@@ -35,6 +35,11 @@ struct VerifyArgs {
     const float* prev_stash;
     const int32_t* prev_accept_len;
     int prev_T;
+    // Gated RMS normalisation of the outputs (NULL norm_z: none): o <- o / sqrt(mean(o^2) + eps)
+    // * norm_w * silu(norm_z) per (token, value head); norm_z has v's layout and dtype.
+    const void* norm_z;
+    const float* norm_w;
+    float norm_eps;
 };
 
 // Arguments of the second phase of a two-phase commit.
@@ -75,6 +80,19 @@ struct ConvArgs {
 // Host launchers; return cudaSuccess or the launch error. Shapes are validated by the caller.
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_short_conv(const ConvArgs& a, int K, bool bf16, cudaStream_t stream);
+
+// Gated RMS normalisation of rows of d elements (gdn_norm.cu). y may be x (in place).
+struct NormArgs {
+    const void* x;       // [rows][d], fp32 or bf16
+    const void* z;       // [rows][d], fp32 or bf16
+    const float* w;      // [d]
+    void* y;             // [rows][d], fp32 or bf16
+    int64_t rows;
+    int d;               // a multiple of 4, <= 4096
+    float eps;
+    bool x_bf16, z_bf16, y_bf16;
+};
+cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);

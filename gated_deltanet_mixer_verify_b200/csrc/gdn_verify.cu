@@ -541,15 +541,34 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);
-    if (head_kernel_applies(a)) return launch_verify_head(a, stream);
-    switch (a.dk) {
-        case 16: return launch_verify_dk<16>(a, stream);
-        case 32: return launch_verify_dk<32>(a, stream);
-        case 64: return launch_verify_dk<64>(a, stream);
-        case 128: return launch_verify_dk<128>(a, stream);
-        default: return cudaErrorInvalidValue;
+    if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);   // fuses the gated norm
+    // Other kernels: the mixer writes o, then the gated norm runs over o in place.
+    VerifyArgs m = a;
+    m.norm_z = nullptr;
+    if (head_kernel_applies(m)) {
+        e = launch_verify_head(m, stream);
+    } else {
+        switch (m.dk) {
+            case 16: e = launch_verify_dk<16>(m, stream); break;
+            case 32: e = launch_verify_dk<32>(m, stream); break;
+            case 64: e = launch_verify_dk<64>(m, stream); break;
+            case 128: e = launch_verify_dk<128>(m, stream); break;
+            default: return cudaErrorInvalidValue;
+        }
     }
+    if (e != cudaSuccess || !a.norm_z) return e;
+    NormArgs n;
+    n.x = a.o;
+    n.z = a.norm_z;
+    n.w = a.norm_w;
+    n.y = a.o;
+    n.rows = (int64_t)a.B * a.T * a.Hv;
+    n.d = a.dv;
+    n.eps = a.norm_eps;
+    n.x_bf16 = a.out_bf16 != 0;
+    n.z_bf16 = a.in_bf16 != 0;
+    n.y_bf16 = a.out_bf16 != 0;
+    return launch_gated_rmsnorm(n, stream);
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream) {

@@ -49,9 +49,11 @@ struct __align__(1024) TcSmem {
     float2 X2[DV][TM];       // (x_s, x_s) per state row: ready-made operands of the packed FMAs
     // Commit-on-next-verify: the previous block's stash for this head as stored (khat'_t rows,
     // scaled in place to KP_t = c_t khat'_t; the decays G'; the u'_t rows), and W = KP [khat;
-    // qhat]^T, the correction of the dots for the committed state.
+    // qhat]^T, the correction of the dots for the committed state. With the gated norm instead
+    // (never both), PS holds the block's gate rows z_t (input dtype) and then the d_v weights.
     float PS[2 * TM * DK + TM];
     float W[TM][NB];
+    float NSS[8][TM / 2];    // gated norm: per warp, its 4 tokens' partial sums of squares
     float Gram[NB][TM];
     float G[TM], Beta[TM], D[TM];
     float A[TM][TM], Cq[TM][TM], Tm[TM][TM], Mo[TM][TM], E[TM][TM];
@@ -137,8 +139,26 @@ __device__ __forceinline__ void commit_rows(const TcSmem& sm, float* dst, int wa
     }
 }
 
+// Gated norm: nw silu(z_t) for this thread's row and its 4 tokens, from the gate rows and
+// weights staged in PS (waits for their copies, bounded; a timeout sets pfail).
+template <typename InT>
+__device__ __forceinline__ void gate_factors(TcSmem& sm, const VerifyArgs& p, int T, int tid, float (&gz)[TM / 2]) {
+    if (!mbar_wait_bounded(&sm.prev_full, 0, kMaxPolls)) sm.pfail = 1;
+    const int row = tid & (DV - 1);
+    const InT* zs = reinterpret_cast<const InT*>(sm.PS);
+    const float nw = reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(sm.PS) +
+                                                    TM * DV * sizeof(InT))[row];
+#pragma unroll
+    for (int tt = 0; tt < TM / 2; ++tt) {
+        const int t = (TM / 2) * (tid >> 7) + tt;
+        const float z = (t < T) ? to_f(zs[t * DV + row]) : 0.f;
+        gz[tt] = nw * __fdividef(z, 1.f + __expf(-z));
+    }
+}
+
 // PRE: commit-on-next-verify (the previous block's stash is applied to the state first).
-template <typename InT, typename OutT, bool PRE>
+// NORM: gated RMS normalisation of the outputs before they are stored.
+template <typename InT, typename OutT, bool PRE, bool NORM>
 __global__ void __launch_bounds__(kThreads, 2)
     gdn_verify_tc_kernel(const __grid_constant__ CUtensorMap smap, const VerifyArgs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -169,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (tid == 128) {
         mbar_init(&sm.full, 1);
         mbar_init(&sm.mma_done, 1);
-        if (precommit) mbar_init(&sm.prev_full, 1);
+        if (precommit || NORM) mbar_init(&sm.prev_full, 1);
         fence_barrier_init();
         mbar_arrive_expect_tx(&sm.full, kTileBytes);
         for (int kb = 0; kb < 4; ++kb) tc::tma_load_2d(&sm.S[kb * DV * 32], &smap, kb * 32, item * DV, &sm.full);
@@ -210,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int t = 0; t < TM; ++t)
         vrow[t] = (t < T) ? ld_in<InT>(p.v, vo_base + t * tok_stride + (tid & (DV - 1))) : 0.f;
+    float gz[TM / 2];   // gated norm: nw silu(z) of this row for its 4 tokens, formed in slack time
     if (warp == 4) {   // tensor memory: one allocation, off the gate chain
         if (lane == 0) {
             sm.fail = 0;
@@ -239,6 +260,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             bulk_prefetch_l2(qb + ((((size_t)nb * T + t) * p.Hk + ng) * DK) * el, (uint32_t)(DK * el));
             bulk_prefetch_l2(kb + ((((size_t)nb * T + t) * p.Hk + ng) * DK) * el, (uint32_t)(DK * el));
             bulk_prefetch_l2(vb + ((((size_t)nb * T + t) * p.Hv + nh) * DV) * el, (uint32_t)(DV * el));
+            if (NORM)   // the gate rows (v's layout)
+                bulk_prefetch_l2(static_cast<const char*>(p.norm_z) + ((((size_t)nb * T + t) * p.Hv + nh) * DV) * el,
+                                 (uint32_t)(DV * el));
         }
     }
 
@@ -383,7 +407,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                                     tc::desc_kmajor_sw128(bb + kb * 2 * NB * 128 + ks * 32), id16, true);
             tc::mma_commit(&sm.mma_done);
         }
+        if (NORM) gate_factors<InT>(sm, p, T, tid, gz);   // tokens 4..7, while the MMAs run
     } else {
+        if (NORM && warp == 3) {
+            // The block's gate rows and the weights into PS (needed only by the last phase): lane
+            // 0 posts the bytes, lanes 0..T-1 copy a row each, lane T the weights. Off the split's
+            // path, after the block barrier that follows the barrier's initialisation.
+            const uint32_t row_bytes = DV * sizeof(InT);
+            if (lane == 0) mbar_arrive_expect_tx(&sm.prev_full, T * row_bytes + DV * 4);
+            __syncwarp();
+            if (lane < T)
+                bulk_g2s(reinterpret_cast<unsigned char*>(sm.PS) + lane * row_bytes,
+                         static_cast<const InT*>(p.norm_z) + vo_base + lane * tok_stride, row_bytes, &sm.prev_full);
+            else if (lane == T)
+                bulk_g2s(reinterpret_cast<unsigned char*>(sm.PS) + TM * row_bytes, p.norm_w, DV * 4, &sm.prev_full);
+        }
         named_sync(3, 256);     // all 16 Gram rows are stored
         // ... the T x T algebra (barrier 1 between steps): the decayed coefficients, one entry
         // per thread, and the commit decays ...
@@ -480,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             sm.W[t][n] = acc;
         }
+        if (NORM) gate_factors<InT>(sm, p, T, tid, gz);   // tokens 0..3 (a shorter path than the split's)
     }
     __syncthreads();
     const int L = sm.L;
@@ -521,18 +560,44 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int s = 0; s < TM; s += 2)
                 *reinterpret_cast<float4*>(&sm.X2[row][s]) = make_float4(xs[s], xs[s], xs[s + 1], xs[s + 1]);
         }
+        // Outputs of tokens 4 hb .. 4 hb + 3 for this row (0 past T).
+        float ovs[TM / 2];
+#pragma unroll
+        for (int tt = 0; tt < TM / 2; ++tt) {
+            const int t = (TM / 2) * hb + tt;
+            float ov = 0.f;
+            if (t < T) {
+                ov = sm.D[t] * (hb ? dots[TM + TM / 2 + tt] : dots[TM + tt]);   // static indices
+#pragma unroll
+                for (int s = 0; s < TM; ++s)
+                    if (s <= t) ov = fmaf(sm.Mo[t][s], xs[s], ov);
+            }
+            ovs[tt] = ov;
+        }
+        if (NORM) {
+            // Each token's 128 outputs sit in the 128 threads of this half (warps 4 hb .. +3):
+            // the warp's four sums of squares by a halving butterfly (token tt ends in lanes
+            // 8 tt .. 8 tt + 7), then the half's four partials (named barrier 5 + hb, which every
+            // thread of the half reaches whatever ok is).
+            float sq[TM / 2];
+#pragma unroll
+            for (int tt = 0; tt < TM / 2; ++tt) sq[tt] = ovs[tt] * ovs[tt];
+            Halve<TM / 2, 16>::run(sq, lane);
+            if ((lane & 7) == 0) sm.NSS[warp][lane >> 3] = sq[0];
+            named_sync(5 + hb, 128);
+#pragma unroll
+            for (int tt = 0; tt < TM / 2; ++tt) {
+                const float tot = sm.NSS[4 * hb][tt] + sm.NSS[4 * hb + 1][tt] + sm.NSS[4 * hb + 2][tt] +
+                                  sm.NSS[4 * hb + 3][tt];
+                ovs[tt] *= rsqrtf(tot / (float)DV + p.norm_eps) * gz[tt];
+            }
+        }
         if (ok) {
             OutT* op = reinterpret_cast<OutT*>(p.o);
 #pragma unroll
             for (int tt = 0; tt < TM / 2; ++tt) {
                 const int t = (TM / 2) * hb + tt;
-                if (t < T) {
-                    float ov = sm.D[t] * (hb ? dots[TM + TM / 2 + tt] : dots[TM + tt]);   // static indices
-#pragma unroll
-                    for (int s = 0; s < TM; ++s)
-                        if (s <= t) ov = fmaf(sm.Mo[t][s], xs[s], ov);
-                    st_out<OutT>(op, vo_base + t * tok_stride + row, ov);
-                }
+                if (t < T) st_out<OutT>(op, vo_base + t * tok_stride + row, ovs[tt]);
             }
             if (p.stash) {
                 float* st = p.stash + head * stash_floats_per_head(T, DK, DV);
@@ -582,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // Drain after a timeout (bounded), then free the tensor memory (always).
     if (!ok && tid == 0) {
         mbar_wait_bounded(&sm.full, 0, kMaxPolls);
-        if (precommit) mbar_wait_bounded(&sm.prev_full, 0, kMaxPolls);
+        if (precommit || NORM) mbar_wait_bounded(&sm.prev_full, 0, kMaxPolls);
         if (!sm.fail) mbar_wait_bounded(&sm.mma_done, 0, kMaxPolls);
     }
     tc::fence_before_sync();
@@ -590,11 +655,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 4) tc::tmem_dealloc(tmem_a, 256);
 }
 
-template <typename InT, typename OutT, bool PRE>
+template <typename InT, typename OutT, bool PRE, bool NORM>
 cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
     constexpr size_t smem = sizeof(TcSmem);
     // Per call: the attribute belongs to the function on the current device.
-    cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT, PRE>,
+    cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT, PRE, NORM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     CUtensorMap map;
@@ -606,13 +671,14 @@ cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     VerifyArgs ap = a;
     ap.prefetch_ahead = 2 * nsm;   // two CTAs per SM are resident
-    gdn_verify_tc_kernel<InT, OutT, PRE><<<a.B * a.Hv, kThreads, smem, stream>>>(map, ap);
+    gdn_verify_tc_kernel<InT, OutT, PRE, NORM><<<a.B * a.Hv, kThreads, smem, stream>>>(map, ap);
     return cudaGetLastError();
 }
 
 template <typename InT, typename OutT>
 cudaError_t launch_tc_pre(const VerifyArgs& a, cudaStream_t stream) {
-    return a.prev_stash ? launch_tc_t<InT, OutT, true>(a, stream) : launch_tc_t<InT, OutT, false>(a, stream);
+    if (a.prev_stash) return launch_tc_t<InT, OutT, true, false>(a, stream);
+    return a.norm_z ? launch_tc_t<InT, OutT, false, true>(a, stream) : launch_tc_t<InT, OutT, false, false>(a, stream);
 }
 
 }  // namespace

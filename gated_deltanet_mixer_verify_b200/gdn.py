@@ -65,9 +65,12 @@ def _load():
     lib.gdn_chunk_prefill_prepare.argtypes = [S, ctypes.c_int32] + [_VP] * 7 + [ctypes.c_size_t, _VP]
     lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
     lib.gdn_short_conv.argtypes = [S, ctypes.c_int32] + [_VP] * 11
+    lib.gdn_verify_step_gated.argtypes = [S] + [_VP] * 12 + [ctypes.c_float] + [_VP] * 3
+    lib.gdn_gated_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int32, _VP, ctypes.c_int32, _VP, ctypes.c_int32,
+                                      _VP, ctypes.c_float, _VP, ctypes.c_int32, _VP]
     for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_commit_and_verify", "gdn_chunk_prefill",
                "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan",
-               "gdn_short_conv"):
+               "gdn_short_conv", "gdn_verify_step_gated", "gdn_gated_rmsnorm"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -190,6 +193,37 @@ def commit_and_verify(q, k, v, a, b, A_log, dt_bias, state, prev_stash, prev_acc
                                          _ptr(prev_accept_len), _ptr(accept_len), _ptr(o), _ptr(stash),
                                          _stream(stream)))
     return o
+
+
+def verify_step_gated(q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept_len, norm_z, norm_w,
+                      norm_eps=1e-6, o=None, stash=None, l2_eps=1e-6, scale=1.0, status_word=None,
+                      out_dtype=torch.float32, stream=None):
+    """verify_step whose outputs are o / sqrt(mean(o^2) + norm_eps) * norm_w * silu(norm_z) per
+    (token, value head); norm_z has v's shape and dtype, norm_w is [d_v] fp32. Returns o."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    if norm_z.shape != v.shape or norm_z.dtype != v.dtype:
+        raise ValueError("norm_z must have v's shape and dtype")
+    if o is None:
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+    _check(_load().gdn_verify_step_gated(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                         _ptr(A_log), _ptr(dt_bias), _ptr(state_in), _ptr(state_out),
+                                         _ptr(accept_len), _ptr(norm_z), _ptr(norm_w), float(norm_eps), _ptr(o),
+                                         _ptr(stash), _stream(stream)))
+    return o
+
+
+def gated_rmsnorm(x, z, w, eps=1e-6, y=None, out_dtype=None, stream=None):
+    """y = x / sqrt(mean(x^2) + eps) * w * silu(z) over the last axis (x, z [..., d]; w [d] fp32).
+    y may be x (in place). Returns y."""
+    d = x.shape[-1]
+    if z.shape != x.shape or w.shape != (d,):
+        raise ValueError("x, z [..., d] and w [d] disagree")
+    if y is None:
+        y = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+    _check(_load().gdn_gated_rmsnorm(x.numel() // d if d else 0, d, _ptr(x), _dtype_code(x.dtype), _ptr(z),
+                                     _dtype_code(z.dtype), _ptr(w), float(eps), _ptr(y), _dtype_code(y.dtype),
+                                     _stream(stream)))
+    return y
 
 
 def conv_channels(H_k, H_v, d_k, d_v) -> int:

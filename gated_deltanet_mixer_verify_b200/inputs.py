@@ -159,6 +159,16 @@ def make_conv_block(w: Workload, K: int = 4, layer: int = 0) -> dict:
     return out
 
 
+def make_norm_inputs(w: Workload, layer: int = 0) -> dict:
+    """Synthetic inputs of the gated output normalisation: the gate z ~ N(0, 1) with v's shape
+    [B, T, H_v, d_v] in the input dtype, and the weight norm_w ~ U(0.5, 1.5) [d_v] fp32. Its own
+    stream, (seed, layer, 9)."""
+    rng = np.random.default_rng([w.seed, layer, 9])
+    z = rng.standard_normal((w.B, w.T, w.H_v, w.d_v), dtype=np.float32)
+    nw = rng.uniform(0.5, 1.5, size=w.d_v).astype(np.float32)
+    return {"norm_z": _store(z, w.in_dtype), "norm_w": torch.from_numpy(nw)}
+
+
 def as_f64(inputs: dict) -> dict:
     """The same inputs as float64 NumPy arrays (exact: every stored value is representable)."""
     out = {}

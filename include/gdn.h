@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 4   /* 4: gdn_short_conv; 3: gdn_commit_and_verify; 2: prefill split into prepare / scan */
+#define GDN_ABI_VERSION 5   /* 5: gated norm; 4: gdn_short_conv; 3: gdn_commit_and_verify; 2: prefill phases */
 
 typedef enum {
     GDN_OK = 0,
@@ -246,6 +246,42 @@ gdn_status gdn_chunk_prefill_noalloc(const gdn_shape* shape, int32_t chunk,
                                      const float* A_log, const float* dt_bias,
                                      const float* state_in, float* state_out, void* o,
                                      void* stream);
+
+/*
+ * gdn_verify_step_gated -- gdn_verify_step with the mixer's output gating and normalisation
+ * ("Lithos-metal: Qwen3.8-27B on 40-core M5 Max", table "GDN mixer": projections, recurrence,
+ * gating and normalisation in one mixer; the formula is the plain reading of it): every output
+ * row (one token of one value head, d_v values) becomes
+ *   o <- o / sqrt(mean(o^2) + norm_eps) * norm_w * silu(norm_z)
+ *   norm_z     [B][T][H_v][d_v] in_dtype (the layout of v): the gate input. Required.
+ *   norm_w     [d_v] fp32, shared by all heads.
+ *   norm_eps   >= 0 (e.g. 1e-6), inside the square root.
+ * Statistics are fp32. The tensor-core verify kernel applies it to its outputs in registers
+ * (one extra read of norm_z); other shapes run the mixer, then gdn_gated_rmsnorm over o in
+ * place (from o as stored in out_dtype). d_v must be a multiple of 4. Everything else is as
+ * gdn_verify_step, whose stash and state are unaffected.
+ */
+gdn_status gdn_verify_step_gated(const gdn_shape* shape,
+                                 const void* q, const void* k, const void* v,
+                                 const void* a, const void* b,
+                                 const float* A_log, const float* dt_bias,
+                                 const float* state_in, float* state_out,
+                                 const int32_t* accept_len,
+                                 const void* norm_z, const float* norm_w, float norm_eps,
+                                 void* o, float* stash, void* stream);
+
+/*
+ * gdn_gated_rmsnorm -- the same gated RMS normalisation as a standalone pass over any mixer
+ * output (decode, prefill): rows of d elements,
+ *   y = x / sqrt(mean(x^2) + eps) * w * silu(z)
+ *   x, z, y    [rows][d] with dtypes x_dtype, z_dtype, y_dtype (GDN_F32 or GDN_BF16);
+ *              y may be x (in place, same dtype) but must not partially overlap it.
+ *   w          [d] fp32.   d: a multiple of 4, up to 4096.   eps >= 0.
+ * One warp per row, statistics in fp32.
+ */
+gdn_status gdn_gated_rmsnorm(int64_t rows, int32_t d, const void* x, int32_t x_dtype,
+                             const void* z, int32_t z_dtype, const float* w, float eps,
+                             void* y, int32_t y_dtype, void* stream);
 
 /*
  * gdn_short_conv -- the causal short convolution in front of the mixer (one filter of conv_k

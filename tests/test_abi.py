@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 4
+    assert lib.gdn_abi_version() == 5
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -169,3 +169,27 @@ def test_short_conv_validates_on_the_host(gdn):
     empty = gdn.make_shape(B=0, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
     assert lib.gdn_short_conv(ctypes.byref(empty), 4, *([None] * 6), None, None, None, None, None) == INVALID
     assert lib.gdn_short_conv(ctypes.byref(empty), 4, *([None] * 5), fake, None, None, None, None, None) == 0
+
+
+def test_gated_norm_entry_points_validate_on_the_host(gdn):
+    INVALID, UNSUP = -1, -2
+    lib = gdn.lib()
+    fake = 0x100000
+    F32, BF16 = 0, 1
+    norm = lambda rows=4, d=128, x=fake, y=0x200000, xt=F32, yt=F32, eps=1e-6: lib.gdn_gated_rmsnorm(
+        rows, d, x, xt, fake, BF16, fake, eps, y, yt, None)
+    assert norm(d=126) == INVALID and "multiple of 4" in lib.gdn_last_error().decode()
+    assert norm(d=8192) == INVALID
+    assert norm(eps=-1.0) == INVALID
+    assert norm(xt=7) == INVALID and "dtype 7" in lib.gdn_last_error().decode()
+    assert norm(y=fake + 16) == INVALID and "partially overlaps" in lib.gdn_last_error().decode()
+    assert norm(y=fake, yt=BF16) == INVALID and "one dtype" in lib.gdn_last_error().decode()
+    assert norm(x=fake + 8) == INVALID and "not 16-byte aligned" in lib.gdn_last_error().decode()
+    assert norm(rows=0, x=None, y=None) == 0
+    sh = gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128)
+    gated = lambda z=fake, w=fake, eps=1e-6, shape=sh: lib.gdn_verify_step_gated(
+        ctypes.byref(shape), *([fake] * 8), None, fake, z, w, eps, fake, None, None)
+    assert gated(z=None) == INVALID and "norm_z is NULL" in lib.gdn_last_error().decode()
+    assert gated(w=None) == INVALID and "norm_w is NULL" in lib.gdn_last_error().decode()
+    assert gated(eps=-1.0) == INVALID
+    assert gated(shape=gdn.make_shape(B=2, T=8, H_k=1, H_v=1, d_k=16, d_v=18)) == UNSUP

@@ -66,3 +66,14 @@ def test_reference_arm_short_conv():
     assert out.returncode == 0, out.stderr[-2000:]
     d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
     assert d["config"]["workload"] == "short_conv" and d["cpu_baseline"]["cores"] == 1 and d["value"] > 0
+
+
+def test_gated_bytes_and_reference_arm(bench):
+    w = workload("batched_verify")
+    assert bench.gated_bytes(w) == bench.algorithmic_bytes(w) + 64 * 8 * 48 * 128 * 2 + 128 * 4
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "verify_gated", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"]["workload"] == "verify_gated" and d["value"] > 0

@@ -376,3 +376,107 @@ void oracle_gated_rmsnorm(int64_t n, int d, const double* o, const double* z, co
         }
     }
 }
+
+/*
+ * Acceptance of a verify block ("Qwen 3.8 27B mac m5: 200 tok/s, audited", section "How does
+ * DSpark speculative decoding create more than one token per read?": up to seven guesses plus
+ * the anchor, exact speculative sampling; greedy mode keeps a guess only if it matches the
+ * large model's token; sampled mode accepts it with probability p / q capped at one, then a
+ * correction token, or a bonus token when every guess was right).
+ *
+ * Per sequence b, tokens[b][0] is the anchor and tokens[b][t] (t = 1 .. T-1) the drafts. Target
+ * row t (logits over V) is the large model's prediction of the token after row t; draft row t
+ * (sampled mode) is the drafter's distribution that proposed tokens[b][t + 1]. With
+ * p_t = softmax(target_t / tau), q_t = softmax(draft_t / tau):
+ *   greedy:  draft t+1 survives iff tokens[t+1] == argmax p_t (lowest index among equal maxima);
+ *   sampled: draft t+1 survives iff u[t+1] * q_t(tokens[t+1]) < p_t(tokens[t+1])
+ *            (u < min(1, p / q) without a division);
+ *   n = the number of leading survivors (0 .. T-1); accept_len = n + 1 (the anchor and the
+ *   surviving drafts: the rows whose state the mixer commits);
+ *   next token: greedy argmax p_n; sampled, n < T-1: drawn from the residual max(0, p_n - q_n)
+ *   (normalised), n = T-1: drawn from p_{T-1}; a draw with u[0] takes the first index j whose
+ *   cumulative mass exceeds u[0] times the total.
+ * target: [B][T][V]; draft: [B][T-1][V] or NULL (greedy); tokens: [B][T]; u: [B][T] or NULL.
+ * Diagnostics (may be NULL): pd, qd [B][T-1] = p_t and q_t at the draft token.
+ */
+static void softmax_row(const double* l, int V, double tau, double* p) {
+    double m = l[0];
+    for (int j = 1; j < V; ++j) m = fmax(m, l[j]);
+    double s = 0.0;
+    for (int j = 0; j < V; ++j) s += exp((l[j] - m) / tau);
+    for (int j = 0; j < V; ++j) p[j] = exp((l[j] - m) / tau) / s;
+}
+
+static int draw(const double* w, int V, double u) {
+    double tot = 0.0;
+    for (int j = 0; j < V; ++j) tot += w[j];
+    const double target = u * tot;
+    double c = 0.0;
+    for (int j = 0; j < V; ++j) {
+        c += w[j];
+        if (c > target && w[j] > 0.0) return j;
+    }
+    for (int j = V - 1; j >= 0; --j)
+        if (w[j] > 0.0) return j;
+    return 0;
+}
+
+int oracle_accept(int B, int T, int V, const double* target, const double* draft, const int32_t* tokens,
+                  const double* u, double tau, int sampled, int32_t* accept_len, int32_t* next_token, double* pd,
+                  double* qd) {
+    if (T < 1 || V < 1 || (sampled && (!draft || !u)) || !(tau > 0.0)) return -1;
+    double* p = (double*)malloc(sizeof(double) * (size_t)V);
+    double* q = (double*)malloc(sizeof(double) * (size_t)V);
+    for (int b = 0; b < B; ++b) {
+        const int32_t* tok = tokens + (int64_t)b * T;
+        int n = 0;
+        int stopped = 0;
+        for (int t = 0; t + 1 < T; ++t) {
+            const double* lt = target + ((int64_t)b * T + t) * V;
+            const int d = tok[t + 1];
+            int ok;
+            if (!sampled) {
+                int am = 0;
+                for (int j = 1; j < V; ++j)
+                    if (lt[j] > lt[am]) am = j;
+                ok = (d == am);
+                if (pd) pd[(int64_t)b * (T - 1) + t] = (double)am;
+            } else {
+                softmax_row(lt, V, tau, p);
+                softmax_row(draft + ((int64_t)b * (T - 1) + t) * V, V, tau, q);
+                const double pv = (d >= 0 && d < V) ? p[d] : 0.0;
+                const double qv = (d >= 0 && d < V) ? q[d] : 0.0;
+                if (pd) pd[(int64_t)b * (T - 1) + t] = pv;
+                if (qd) qd[(int64_t)b * (T - 1) + t] = qv;
+                ok = u[(int64_t)b * T + t + 1] * qv < pv;
+            }
+            if (!stopped && ok) {
+                ++n;
+            } else {
+                stopped = 1;
+            }
+        }
+        accept_len[b] = n + 1;
+        const double* ln = target + ((int64_t)b * T + n) * V;
+        if (!sampled) {
+            int am = 0;
+            for (int j = 1; j < V; ++j)
+                if (ln[j] > ln[am]) am = j;
+            next_token[b] = am;
+        } else {
+            softmax_row(ln, V, tau, p);
+            if (n < T - 1) {
+                softmax_row(draft + ((int64_t)b * (T - 1) + n) * V, V, tau, q);
+                for (int j = 0; j < V; ++j) q[j] = fmax(p[j] - q[j], 0.0);
+                double tot = 0.0;
+                for (int j = 0; j < V; ++j) tot += q[j];
+                next_token[b] = draw(tot > 0.0 ? q : p, V, u[(int64_t)b * T]);
+            } else {
+                next_token[b] = draw(p, V, u[(int64_t)b * T]);
+            }
+        }
+    }
+    free(p);
+    free(q);
+    return 0;
+}

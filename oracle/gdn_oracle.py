@@ -48,6 +48,9 @@ def _load():
         lib.oracle_short_conv.restype = ctypes.c_int
         lib.oracle_gated_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int, _D, _D, _D, ctypes.c_double, _D]
         lib.oracle_gated_rmsnorm.restype = None
+        lib.oracle_accept.argtypes = [ctypes.c_int] * 3 + [_D, _D, _I32, _D, ctypes.c_double, ctypes.c_int,
+                                                           _I32, _I32, _D, _D]
+        lib.oracle_accept.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -214,3 +217,26 @@ def gated_rmsnorm(o, z, w, eps=1e-6):
     y = np.empty_like(o)
     _load().oracle_gated_rmsnorm(o.size // d if d else 0, d, _p(o), _p(z), _p(w), float(eps), _p(y))
     return y
+
+
+def accept(target, tokens, draft=None, u=None, tau=1.0, sampled=False):
+    """Acceptance of verify blocks (oracle_accept).
+
+    target: [B, T, V] logits; tokens: [B, T] int (row 0 the anchor); draft: [B, T-1, V] logits
+    and u: [B, T] uniforms in sampled mode. Returns (accept_len [B], next_token [B], pd, qd):
+    pd / qd [B, T-1] are p_t and q_t at each draft token (greedy: pd holds the argmax).
+    """
+    target = _f64(target)
+    B, T, V = target.shape
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    d = None if draft is None else _f64(draft)
+    uu = None if u is None else _f64(u)
+    L = np.zeros(B, dtype=np.int32)
+    nt = np.zeros(B, dtype=np.int32)
+    pd = np.zeros((B, max(T - 1, 1)))
+    qd = np.zeros((B, max(T - 1, 1)))
+    rc = _load().oracle_accept(B, T, V, _p(target), _p(d), _pi(tok), _p(uu), float(tau), int(bool(sampled)),
+                               _pi(L), _pi(nt), _p(pd), _p(qd))
+    if rc != 0:
+        raise ValueError("oracle_accept: bad arguments")
+    return L, nt, pd[:, :T - 1], qd[:, :T - 1]

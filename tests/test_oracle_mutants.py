@@ -1,5 +1,5 @@
 """Plant plausible mistakes in copies of the oracle's C source and check that the pins in
-test_oracle.py, test_oracle_conv.py and test_oracle_norm.py catch every one (a dropped term, a wrong sign or index,
+test_oracle*.py catch every one (a dropped term, a wrong sign or index,
 a transposed operand, an off-by-one commit, reversed filter taps, a history not rewound). Mistakes are planted only in the oracle, on the CPU."""
 import os
 import subprocess
@@ -47,16 +47,27 @@ MUTANTS = {
                                    "const double g = 1.0 / (1.0 + exp(-zrow[j]));"),
     "norm_weight_dropped": ("y[r * d + j] = orow[j] * inv * w[j] * g;", "y[r * d + j] = orow[j] * inv * g;"),
     "norm_gate_on_wrong_row": ("const double* zrow = z + r * d;", "const double* zrow = z;"),
+    "accept_ratio_inverted": ("ok = u[(int64_t)b * T + t + 1] * qv < pv;", "ok = u[(int64_t)b * T + t + 1] * pv < qv;"),
+    "accept_residual_reversed": ("q[j] = fmax(p[j] - q[j], 0.0);", "q[j] = fmax(q[j] - p[j], 0.0);"),
+    "accept_len_without_anchor": ("accept_len[b] = n + 1;", "accept_len[b] = n;"),
+    "accept_greedy_tie_to_last": ("if (lt[j] > lt[am]) am = j;", "if (lt[j] >= lt[am]) am = j;"),
+    "accept_next_from_previous_row": ("const double* ln = target + ((int64_t)b * T + n) * V;",
+                                      "const double* ln = target + ((int64_t)b * T + (n > 0 ? n - 1 : 0)) * V;"),
+    "accept_temperature_ignored": ("for (int j = 0; j < V; ++j) p[j] = exp((l[j] - m) / tau) / s;",
+                                   "for (int j = 0; j < V; ++j) p[j] = exp(l[j] - m) / s;"),
+    "accept_continues_after_rejection": ("if (!stopped && ok) {", "if (ok) {"),
 }
 
 
 def pin_file(name):
     """The pins of the function a mutant breaks: conv_* the short convolution's, norm_* the
-    gated normalisation's, the rest the mixer's."""
+    gated normalisation's, accept_* the acceptance's, the rest the mixer's."""
     if name.startswith("conv_"):
         return "test_oracle_conv.py"
     if name.startswith("norm_"):
         return "test_oracle_norm.py"
+    if name.startswith("accept_"):
+        return "test_oracle_accept.py"
     return "test_oracle.py"
 
 

@@ -563,6 +563,63 @@ gdn_status gdn_short_conv(const gdn_shape* shape, int32_t conv_k, const void* q,
                     who);
 }
 
+static gdn_status check_accept(const gdn_accept_shape* s, const char* who) {
+    if (!s) return fail(GDN_ERR_INVALID_ARG, "%s: shape is NULL", who);
+    if (s->B < 0 || s->T < 1 || s->V < 1)
+        return fail(GDN_ERR_INVALID_ARG, "%s: sizes must be positive (B may be 0)", who);
+    if (s->T > 16) return fail(GDN_ERR_UNSUPPORTED, "%s: T %d > 16", who, s->T);
+    if (s->V % 8 != 0 || s->V > (1 << 24))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: V must be a multiple of 8 up to 2^24 (got %d)", who, s->V);
+    if (s->B > (1 << 20)) return fail(GDN_ERR_UNSUPPORTED, "%s: B > 2^20", who);
+    if (s->logits_dtype != GDN_F32 && s->logits_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "%s: logits_dtype %d unknown", who, s->logits_dtype);
+    if (s->sampled != 0 && s->sampled != 1) return fail(GDN_ERR_INVALID_ARG, "%s: sampled must be 0 or 1", who);
+    if (s->sampled && !(s->temperature > 0.f))
+        return fail(GDN_ERR_INVALID_ARG, "%s: temperature must be > 0", who);
+    return GDN_OK;
+}
+
+size_t gdn_accept_workspace_bytes(const gdn_accept_shape* shape) {
+    if (check_accept(shape, "gdn_accept_workspace_bytes") != GDN_OK) return 0;
+    return gdn::accept_workspace_bytes(shape->B, shape->T, shape->V, shape->sampled != 0);
+}
+
+gdn_status gdn_accept(const gdn_accept_shape* shape, const void* target_logits, const void* draft_logits,
+                      const int32_t* tokens, const float* uniforms, int32_t* accept_len, int32_t* next_token,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    const char* who = "gdn_accept";
+    gdn_status st = check_accept(shape, who);
+    if (st != GDN_OK) return st;
+    if (shape->B == 0) return ok();
+    REQUIRE_PTR(target_logits, who);
+    REQUIRE_PTR(tokens, who);
+    REQUIRE_PTR(accept_len, who);
+    REQUIRE_PTR(next_token, who);
+    if (shape->sampled) {
+        if (shape->T > 1) REQUIRE_PTR(draft_logits, who);
+        REQUIRE_PTR(uniforms, who);
+    }
+    const size_t need = gdn::accept_workspace_bytes(shape->B, shape->T, shape->V, shape->sampled != 0);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
+    if (!aligned16(workspace)) return fail(GDN_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", who);
+    gdn::AcceptArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = shape->B;
+    a.T = shape->T;
+    a.V = shape->V;
+    a.bf16 = shape->logits_dtype == GDN_BF16;
+    a.sampled = shape->sampled != 0;
+    a.tau = shape->sampled ? shape->temperature : 1.f;
+    a.target = target_logits;
+    a.draft = draft_logits;
+    a.tokens = tokens;
+    a.u = uniforms;
+    a.accept_len = accept_len;
+    a.next_token = next_token;
+    return launched(gdn::launch_accept(a, workspace, static_cast<cudaStream_t>(stream)), who);
+}
+
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
 
 }  // extern "C"

@@ -1,0 +1,366 @@
+// gdn_accept.cu -- device-side acceptance of a verify block: greedy matching or exact
+// speculative sampling, producing the accept counts the mixer commits at and the next token,
+// so that verify -> accept -> commit stays on the GPU.
+//
+// Rule ("Qwen 3.8 27B mac m5: 200 tok/s, audited", section "How does DSpark speculative
+// decoding create more than one token per read?"): row 0 of a block is the anchor, rows
+// 1..T-1 the drafts. Greedy keeps draft t+1 only if it is the target's argmax at row t
+// (lowest index among equal maxima); sampled mode keeps it when u * q_t(d) < p_t(d), i.e. with
+// probability min(1, p / q), p_t = softmax(target_t / tau), q_t = softmax(draft_t / tau). After
+// n leading survivors: accept_len = n + 1; the next token is argmax p_n (greedy), else a draw
+// with u_0 from the residual max(0, p_n - q_n) (n < T-1) or from p_{T-1} (all survived).
+//
+// Kernel 1 (one CTA per logit row, target rows then draft rows): streams the row once with
+// 16-byte loads, keeping the maximum and its first index (greedy) or the online maximum and
+// sum of 2^(x log2(e) / tau - max) (sampled). The last CTA to finish a sequence's rows (a
+// fence, then an atomic counter: nobody waits) finds n and writes accept_len (and the greedy
+// next token). Kernel 2 (sampled; 8 CTAs per sequence): tile sums (256 logits a tile) of the
+// residual over row n; the last CTA of the sequence draws the token by inverse CDF, first over
+// the tile sums, then inside one tile with a warp scan. Both are HBM-bound.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn_device.cuh"
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+using namespace dev;
+
+constexpr int kRowThreads = 512;
+constexpr int kTile = 256;         // logits per tile of the residual draw (8 per lane of a warp)
+constexpr int kSplit = 8;          // CTAs per sequence in the residual pass
+constexpr int kSplitThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+using RowStat = AcceptRowStat;
+
+template <typename T>
+__device__ __forceinline__ void ld8l(const T* p, float (&x)[8]);
+template <>
+__device__ __forceinline__ void ld8l<float>(const float* p, float (&x)[8]) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(p)), b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void ld8l<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        x[2 * e] = __uint_as_float(w[e] << 16);
+        x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float ld1l(const T* p, int64_t i) {
+    return to_f(p[i]);
+}
+
+// (value, index) maximum with ties to the lower index.
+__device__ __forceinline__ void better(float& v, int& i, float v2, int i2) {
+    if (v2 > v || (v2 == v && i2 < i)) {
+        v = v2;
+        i = i2;
+    }
+}
+
+// Online (max, sum) of base-2 exponentials: merge (m2, s2) into (m, s).
+__device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2) {
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;
+    s = s * exp2_approx(m - mn) + s2 * exp2_approx(m2 - mn);
+    m = mn;
+}
+
+// p_t(d) and q_t(d) from the statistics; the acceptance decisions and n of sequence b.
+template <typename LT>
+__device__ int leading_run(const AcceptArgs& a, const RowStat* st, int b) {
+    const LT* tg = static_cast<const LT*>(a.target);
+    const LT* dr = static_cast<const LT*>(a.draft);
+    const float c = kLog2e / a.tau;
+    int n = 0;
+    for (int t = 0; t + 1 < a.T; ++t) {
+        const int d = a.tokens[(int64_t)b * a.T + t + 1];
+        bool ok;
+        if (!a.sampled) {
+            ok = d == __ldcg(&st[(int64_t)b * a.T + t].arg);
+        } else if (d < 0 || d >= a.V) {
+            ok = false;
+        } else {
+            const RowStat sp = {__ldcg(&st[(int64_t)b * a.T + t].m), __ldcg(&st[(int64_t)b * a.T + t].s), 0, 0};
+            const int64_t qr = (int64_t)a.B * a.T + (int64_t)b * (a.T - 1) + t;
+            const RowStat sq = {__ldcg(&st[qr].m), __ldcg(&st[qr].s), 0, 0};
+            const float p = exp2_approx(ld1l(tg, ((int64_t)b * a.T + t) * a.V + d) * c - sp.m) / sp.s;
+            const float q = exp2_approx(ld1l(dr, ((int64_t)b * (a.T - 1) + t) * a.V + d) * c - sq.m) / sq.s;
+            ok = a.u[(int64_t)b * a.T + t + 1] * q < p;
+        }
+        if (!ok) break;
+        ++n;
+    }
+    return n;
+}
+
+template <typename LT>
+__global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const AcceptArgs a) {
+    const int64_t r = blockIdx.x;
+    const int64_t ntarget = (int64_t)a.B * a.T;
+    const LT* row = r < ntarget ? static_cast<const LT*>(a.target) + r * a.V
+                                : static_cast<const LT*>(a.draft) + (r - ntarget) * a.V;
+    const int b = r < ntarget ? (int)(r / a.T) : (int)((r - ntarget) / (a.T - 1));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float c = kLog2e / a.tau;
+    float m = -INFINITY, s = 0.f;
+    int arg = 0x7fffffff;
+    // Four 8-logit groups in flight per thread.
+    for (int base = 8 * tid; base < a.V; base += 4 * 8 * kRowThreads) {
+        float x[4][8];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int i = base + g * 8 * kRowThreads;
+            if (i < a.V) {
+                ld8l<LT>(row + i, x[g]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[g][e] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int i = base + g * 8 * kRowThreads;
+            if (!a.sampled) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (x[g][e] > m) {   // indices rise within a thread: strict > keeps the first
+                        m = x[g][e];
+                        arg = i + e;
+                    }
+            } else {
+                float lm = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[g][e] * c);
+                if (lm > -INFINITY) {
+                    float ls = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ls += exp2_approx(x[g][e] * c - lm);
+                    merge_ms(m, s, lm, ls);
+                }
+            }
+        }
+    }
+    __shared__ float red_m[kRowThreads / 32], red_s[kRowThreads / 32];
+    __shared__ int red_i[kRowThreads / 32];
+    __shared__ bool last;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float m2 = __shfl_xor_sync(kFull, m, off);
+        const float s2 = __shfl_xor_sync(kFull, s, off);
+        const int i2 = __shfl_xor_sync(kFull, arg, off);
+        if (!a.sampled) better(m, arg, m2, i2);
+        else merge_ms(m, s, m2, s2);
+    }
+    if (lane == 0) {
+        red_m[warp] = m;
+        red_s[warp] = s;
+        red_i[warp] = arg;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int w = 1; w < kRowThreads / 32; ++w) {
+            if (!a.sampled) better(m, arg, red_m[w], red_i[w]);
+            else merge_ms(m, s, red_m[w], red_s[w]);
+        }
+        RowStat* st = a.stats + r;
+        st->m = m;
+        st->s = s;
+        st->arg = arg;
+        __threadfence();   // the statistics are visible before this row is counted
+        const int rows_per_seq = a.sampled ? 2 * a.T - 1 : a.T;
+        last = atomicAdd(&a.counters[b], 1) == rows_per_seq - 1;
+    }
+    __syncthreads();
+    if (!last || tid != 0) return;
+    // The last row of sequence b: every row's statistics are in place.
+    __threadfence();
+    const int n = leading_run<LT>(a, a.stats, b);
+    a.accept_len[b] = n + 1;
+    a.nsurv[b] = n;
+    if (!a.sampled) a.next_token[b] = __ldcg(&a.stats[(int64_t)b * a.T + n].arg);
+}
+
+// Residual (or target) weight of logit j of sequence b's row n, from the statistics.
+template <typename LT>
+__device__ __forceinline__ void weights8(const AcceptArgs& a, const LT* pr, const LT* qr, int j, float pm, float ps,
+                                         float qm, float qs, float (&w)[8]) {
+    const float c = kLog2e / a.tau;
+    float x[8];
+    ld8l<LT>(pr + j, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e] = exp2_approx(x[e] * c - pm) / ps;
+    if (qr) {
+        float y[8];
+        ld8l<LT>(qr + j, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = fmaxf(w[e] - exp2_approx(y[e] * c - qm) / qs, 0.f);
+    }
+}
+
+// grid (B, kSplit): tile sums of row n's residual; the last CTA of the sequence draws.
+template <typename LT>
+__global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const AcceptArgs a) {
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = __ldcg(&a.nsurv[b]);
+    const int64_t prow = (int64_t)b * a.T + n;
+    const LT* pr = static_cast<const LT*>(a.target) + prow * a.V;
+    const LT* qr = nullptr;
+    float qm = 0.f, qs = 1.f;
+    if (n < a.T - 1) {
+        const int64_t q = (int64_t)a.B * a.T + (int64_t)b * (a.T - 1) + n;
+        qr = static_cast<const LT*>(a.draft) + ((int64_t)b * (a.T - 1) + n) * a.V;
+        qm = __ldcg(&a.stats[q].m);
+        qs = __ldcg(&a.stats[q].s);
+    }
+    const float pm = __ldcg(&a.stats[prow].m), ps = __ldcg(&a.stats[prow].s);
+    const int ntiles = (a.V + kTile - 1) / kTile;
+    float* tsum = a.tiles + (int64_t)b * ntiles;
+    // Tiles blockIdx.y, +kSplit, ... ; a warp per tile, 8 logits per lane.
+    for (int tile = blockIdx.y + kSplit * warp; tile < ntiles; tile += kSplit * (kSplitThreads / 32)) {
+        const int j = tile * kTile + 8 * lane;
+        float acc = 0.f;
+        if (j < a.V) {
+            float w[8];
+            weights8<LT>(a, pr, qr, j, pm, ps, qm, qs, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc += w[e];
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) tsum[tile] = acc;
+    }
+    __shared__ bool last;
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        last = atomicAdd(&a.counters[a.B + b], 1) == kSplit - 1;
+    }
+    __syncthreads();
+    if (!last || warp != 0) return;
+    __threadfence();
+    // Warp 0 of the last CTA: the total and the tile holding u_0 * total (lane L covers a
+    // contiguous range of tiles), then the logit inside that tile.
+    const int per = (ntiles + 31) / 32;
+    const int t0 = lane * per, t1 = min(t0 + per, ntiles);
+    float mine = 0.f;
+    for (int t = t0; t < t1; ++t) mine += __ldcg(&tsum[t]);
+    float incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const float total = __shfl_sync(kFull, incl, 31);
+    const float target = a.u[(int64_t)b * a.T] * total;
+    const unsigned hit = __ballot_sync(kFull, incl > target && mine > 0.f);
+    const bool fallback = hit == 0;   // warp-uniform
+    int tile = -1;
+    float before = 0.f;
+    if (!fallback) {
+        const int L = __ffs(hit) - 1;
+        if (lane == L) {
+            float cum = incl - mine;
+            for (int t = t0; t < t1; ++t) {
+                const float v = __ldcg(&tsum[t]);
+                if (cum + v > target && v > 0.f) {
+                    tile = t;
+                    break;
+                }
+                cum += v;
+            }
+            if (tile < 0) {   // rounding: the last positive tile of the range
+                for (int t = t1 - 1; t >= t0; --t)
+                    if (__ldcg(&tsum[t]) > 0.f) {
+                        tile = t;
+                        break;
+                    }
+            }
+            before = cum;
+        }
+        tile = __shfl_sync(kFull, tile, L);
+        before = __shfl_sync(kFull, before, L);
+    } else {   // rounding at the very end: the last tile with mass
+        int lt = -1;
+        for (int t = ntiles - 1 - lane; t >= 0; t -= 32)
+            if (__ldcg(&tsum[t]) > 0.f) {
+                lt = t;
+                break;
+            }
+        tile = __reduce_max_sync(kFull, lt);   // its last positive logit is taken below
+    }
+    if (tile < 0) {
+        if (lane == 0) a.next_token[b] = 0;
+        return;
+    }
+    const int j = tile * kTile + 8 * lane;
+    float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (j < a.V) weights8<LT>(a, pr, qr, j, pm, ps, qm, qs, w);
+    float mine2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mine2 += w[e];
+    float incl2 = mine2;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(kFull, incl2, off);
+        if (lane >= off) incl2 += y;
+    }
+    // The first logit whose running mass passes the target; otherwise the tile's last positive.
+    int found = 0x7fffffff, lastpos = -1;
+    float cum = before + incl2 - mine2;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        cum += w[e];
+        if (w[e] > 0.f) {
+            if (cum > target && found == 0x7fffffff) found = j + e;
+            lastpos = j + e;
+        }
+    }
+    const int first = __reduce_min_sync(kFull, found);
+    const int lastp = __reduce_max_sync(kFull, lastpos);
+    if (lane == 0) a.next_token[b] = (!fallback && first != 0x7fffffff) ? first : (lastp >= 0 ? lastp : 0);
+}
+
+}  // namespace
+
+size_t accept_workspace_bytes(int B, int T, int V, bool sampled) {
+    const size_t rows = (size_t)B * T + (sampled ? (size_t)B * (T - 1) : 0);
+    const size_t ntiles = ((size_t)V + kTile - 1) / kTile;
+    return rows * sizeof(RowStat) + (size_t)B * 4 /* nsurv */ + (size_t)2 * B * 4 /* counters */ +
+           (sampled ? (size_t)B * ntiles * 4 : 0) + 64;
+}
+
+cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream) {
+    // Workspace: statistics, then n per sequence, the counters, the tile sums.
+    unsigned char* w = static_cast<unsigned char*>(workspace);
+    const size_t rows = (size_t)a.B * a.T + (a.sampled ? (size_t)a.B * (a.T - 1) : 0);
+    a.stats = reinterpret_cast<RowStat*>(w);
+    w += rows * sizeof(RowStat);
+    a.nsurv = reinterpret_cast<int*>(w);
+    w += (size_t)a.B * 4;
+    a.counters = reinterpret_cast<int*>(w);
+    w += (size_t)2 * a.B * 4;
+    a.tiles = reinterpret_cast<float*>(w);
+    cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)2 * a.B * 4, stream);
+    if (e != cudaSuccess) return e;
+    if (a.bf16) gdn_accept_rows_kernel<__nv_bfloat16><<<(unsigned)rows, kRowThreads, 0, stream>>>(a);
+    else gdn_accept_rows_kernel<float><<<(unsigned)rows, kRowThreads, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !a.sampled) return e;
+    const dim3 grid(a.B, kSplit);
+    if (a.bf16) gdn_accept_draw_kernel<__nv_bfloat16><<<grid, kSplitThreads, 0, stream>>>(a);
+    else gdn_accept_draw_kernel<float><<<grid, kSplitThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

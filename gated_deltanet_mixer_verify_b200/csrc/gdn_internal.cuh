@@ -94,6 +94,32 @@ struct NormArgs {
 };
 cudaError_t launch_gated_rmsnorm(const NormArgs& a, cudaStream_t stream);
 
+// Device-side acceptance of a verify block (gdn_accept.cu).
+struct AcceptRowStat {
+    float m;     // greedy: the row's maximum logit; sampled: max of logit log2(e) / tau
+    float s;     // sampled: sum of 2^(logit log2(e) / tau - m)
+    int arg;     // greedy: first index of the maximum
+    int pad;
+};
+struct AcceptArgs {
+    int B, T, V;
+    bool bf16, sampled;
+    float tau;
+    const void* target;          // [B][T][V]
+    const void* draft;           // [B][T-1][V] (sampled)
+    const int32_t* tokens;       // [B][T]: the anchor, then the drafts
+    const float* u;              // [B][T] (sampled): u[0] for the draw, u[t+1] for draft t+1
+    int32_t* accept_len;         // [B] out
+    int32_t* next_token;         // [B] out
+    int32_t* status_word;
+    AcceptRowStat* stats;        // set by the launcher from the workspace
+    int* nsurv;
+    int* counters;
+    float* tiles;
+};
+size_t accept_workspace_bytes(int B, int T, int V, bool sampled);
+cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream);
+
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);
 

@@ -39,6 +39,12 @@ class _Shape(ctypes.Structure):
                 ("status_word", ctypes.c_void_p)]
 
 
+class _AcceptShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("V", ctypes.c_int32),
+                ("logits_dtype", ctypes.c_int32), ("sampled", ctypes.c_int32),
+                ("temperature", ctypes.c_float)]
+
+
 _lib = None
 _VP = ctypes.c_void_p
 
@@ -65,12 +71,16 @@ def _load():
     lib.gdn_chunk_prefill_prepare.argtypes = [S, ctypes.c_int32] + [_VP] * 7 + [ctypes.c_size_t, _VP]
     lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
     lib.gdn_short_conv.argtypes = [S, ctypes.c_int32] + [_VP] * 11
+    A = ctypes.POINTER(_AcceptShape)
+    lib.gdn_accept.argtypes = [A] + [_VP] * 7 + [ctypes.c_size_t, _VP]
+    lib.gdn_accept_workspace_bytes.argtypes = [A]
+    lib.gdn_accept_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_verify_step_gated.argtypes = [S] + [_VP] * 12 + [ctypes.c_float] + [_VP] * 3
     lib.gdn_gated_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int32, _VP, ctypes.c_int32, _VP, ctypes.c_int32,
                                       _VP, ctypes.c_float, _VP, ctypes.c_int32, _VP]
     for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_commit_and_verify", "gdn_chunk_prefill",
                "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan",
-               "gdn_short_conv", "gdn_verify_step_gated", "gdn_gated_rmsnorm"):
+               "gdn_short_conv", "gdn_verify_step_gated", "gdn_gated_rmsnorm", "gdn_accept"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -224,6 +234,37 @@ def gated_rmsnorm(x, z, w, eps=1e-6, y=None, out_dtype=None, stream=None):
                                      _dtype_code(z.dtype), _ptr(w), float(eps), _ptr(y), _dtype_code(y.dtype),
                                      _stream(stream)))
     return y
+
+
+def _accept_shape(B, T, V, dtype, sampled, temperature) -> _AcceptShape:
+    return _AcceptShape(B, T, V, _dtype_code(dtype), int(bool(sampled)), float(temperature))
+
+
+def accept_workspace_bytes(B, T, V, sampled, dtype=torch.bfloat16) -> int:
+    """Bytes of workspace :func:`accept` needs."""
+    sh = _accept_shape(B, T, V, dtype, sampled, 1.0)
+    return int(_load().gdn_accept_workspace_bytes(ctypes.byref(sh)))
+
+
+def accept(target, tokens, draft=None, uniforms=None, temperature=1.0, workspace=None, accept_len=None,
+           next_token=None, stream=None):
+    """Device-side acceptance of verify blocks. target [B, T, V] logits (bf16 or fp32), tokens
+    [B, T] int32 (the anchor, then the drafts); sampled mode when draft [B, T-1, V] and uniforms
+    [B, T] fp32 are given, greedy otherwise. Returns (accept_len [B], next_token [B]) int32."""
+    B, T, V = target.shape
+    sampled = uniforms is not None
+    sh = _accept_shape(B, T, V, target.dtype, sampled, temperature)
+    if workspace is None:
+        workspace = torch.empty(max(accept_workspace_bytes(B, T, V, sampled, target.dtype), 16),
+                                dtype=torch.uint8, device=target.device)
+    if accept_len is None:
+        accept_len = torch.empty(B, dtype=torch.int32, device=target.device)
+    if next_token is None:
+        next_token = torch.empty(B, dtype=torch.int32, device=target.device)
+    _check(_load().gdn_accept(ctypes.byref(sh), _ptr(target), _ptr(draft), _ptr(tokens), _ptr(uniforms),
+                              _ptr(accept_len), _ptr(next_token), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)))
+    return accept_len, next_token
 
 
 def conv_channels(H_k, H_v, d_k, d_v) -> int:

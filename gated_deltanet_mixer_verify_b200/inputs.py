@@ -169,6 +169,30 @@ def make_norm_inputs(w: Workload, layer: int = 0) -> dict:
     return {"norm_z": _store(z, w.in_dtype), "norm_w": torch.from_numpy(nw)}
 
 
+def make_accept_inputs(w: Workload, V: int = 151936, layer: int = 0, plant: float = 0.8,
+                       dtype: Optional[str] = None) -> dict:
+    """Synthetic acceptance inputs for blocks of workload ``w`` (B sequences of T rows) over a
+    vocabulary of V: target logits ~ N(0, 1) [B, T, V]; draft logits = the target's first T-1
+    rows + N(0, 0.5) noise; tokens [B, T] uniform over V (row 0 the anchor); uniforms [B, T] ~
+    U[0, 1). At a fraction `plant` of the draft positions, both models get +8 on the drafted
+    token's logit (so that acceptance runs look like a real drafter's). Logits are stored in
+    `dtype` (default the workload's input dtype). Its own stream, (seed, layer, 10)."""
+    rng = np.random.default_rng([w.seed, layer, 10])
+    B, T = w.B, w.T
+    f32 = np.float32
+    target = rng.standard_normal((B, T, V), dtype=f32)
+    draft = target[:, :T - 1] + f32(0.5) * rng.standard_normal((B, T - 1, V), dtype=f32)
+    tokens = rng.integers(0, V, size=(B, T)).astype(np.int32)
+    planted = rng.random((B, T - 1)) < plant
+    bi, ti = np.nonzero(planted)
+    target[bi, ti, tokens[bi, ti + 1]] += f32(8.0)
+    draft[bi, ti, tokens[bi, ti + 1]] += f32(8.0)
+    u = rng.random((B, T)).astype(f32)
+    dt = dtype or w.in_dtype
+    return {"target": _store(target, dt), "draft": _store(draft, dt), "tokens": torch.from_numpy(tokens),
+            "uniforms": torch.from_numpy(u)}
+
+
 def as_f64(inputs: dict) -> dict:
     """The same inputs as float64 NumPy arrays (exact: every stored value is representable)."""
     out = {}

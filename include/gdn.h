@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 5   /* 5: gated norm; 4: gdn_short_conv; 3: gdn_commit_and_verify; 2: prefill phases */
+#define GDN_ABI_VERSION 6   /* 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
 
 typedef enum {
     GDN_OK = 0,
@@ -315,6 +315,45 @@ gdn_status gdn_short_conv(const gdn_shape* shape, int32_t conv_k,
                           const void* q, const void* k, const void* v, const float* conv_w,
                           const void* hist_in, void* hist_out, const int32_t* accept_len,
                           void* q_out, void* k_out, void* v_out, void* stream);
+
+/*
+ * gdn_accept -- device-side acceptance of verify blocks, so that verify -> accept -> commit
+ * never leaves the GPU ("Lithos-metal: Qwen3.8-27B on 40-core M5 Max", runtime paragraph on
+ * GPU-resident commit / rollback; "Qwen 3.8 27B mac m5: 200 tok/s, audited", section "How does
+ * DSpark speculative decoding create more than one token per read?": exact speculative
+ * sampling, greedy or sampled, then a correction or a bonus token).
+ *   tokens          [B][T] int32: row 0 the anchor (the last confirmed token), rows 1..T-1 drafts.
+ *   target_logits   [B][T][V] logits_dtype: row t is the large model's prediction of the token
+ *                   after row t.
+ *   draft_logits    [B][T-1][V] logits_dtype (sampled mode; NULL for greedy): row t is the
+ *                   drafter's prediction that proposed draft t+1.
+ *   uniforms        [B][T] fp32 in [0, 1) (sampled mode; NULL for greedy): uniforms[b][t+1]
+ *                   decides draft t+1, uniforms[b][0] draws the next token.
+ *   accept_len      [B] int32 out: 1 + the number of leading drafts that survive (1..T): the
+ *                   block rows the mixer commits (its accept_len argument, on the device).
+ *   next_token      [B] int32 out: greedy, the argmax at row n (the first rejected row, or the
+ *                   last row); sampled, a draw with uniforms[b][0] from max(0, p_n - q_n)
+ *                   normalised (a rejection) or from p_{T-1} (every draft survived).
+ * p_t = softmax(target_t / temperature), q_t = softmax(draft_t / temperature). Greedy keeps
+ * draft t+1 iff it is the first index of the maximum of target row t; sampled keeps it iff
+ * uniforms[b][t+1] * q_t(d) < p_t(d). Decisions are taken in fp32. A draw takes the first index
+ * whose running mass exceeds u times the total. workspace: gdn_accept_workspace_bytes, 16-byte
+ * aligned, contents irrelevant (the call zeroes what it needs). V a multiple of 8, up to 2^24;
+ * T 1..16.
+ */
+typedef struct {
+    int32_t B, T, V;
+    int32_t logits_dtype;    /* GDN_F32 or GDN_BF16, for both logit arrays */
+    int32_t sampled;         /* 0: greedy; 1: exact speculative sampling */
+    float temperature;       /* > 0 (sampled mode) */
+} gdn_accept_shape;
+
+gdn_status gdn_accept(const gdn_accept_shape* shape, const void* target_logits, const void* draft_logits,
+                      const int32_t* tokens, const float* uniforms, int32_t* accept_len, int32_t* next_token,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace gdn_accept needs (0 for an invalid shape). */
+size_t gdn_accept_workspace_bytes(const gdn_accept_shape* shape);
 
 /* Bytes of stash gdn_verify_step writes for this shape (0 for an invalid shape). */
 size_t gdn_stash_bytes(const gdn_shape* shape);

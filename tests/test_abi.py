@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 5
+    assert lib.gdn_abi_version() == 6
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -193,3 +193,23 @@ def test_gated_norm_entry_points_validate_on_the_host(gdn):
     assert gated(w=None) == INVALID and "norm_w is NULL" in lib.gdn_last_error().decode()
     assert gated(eps=-1.0) == INVALID
     assert gated(shape=gdn.make_shape(B=2, T=8, H_k=1, H_v=1, d_k=16, d_v=18)) == UNSUP
+
+
+def test_accept_validates_on_the_host(gdn):
+    INVALID, UNSUP, WORKSPACE = -1, -2, -4
+    lib = gdn.lib()
+    fake = 0x100000
+    need = gdn.accept_workspace_bytes(64, 8, 151936, True)
+    # statistics (16 bytes a row: 8 target + 7 draft rows per sequence), n, two counters, tile sums
+    assert need == 64 * 15 * 16 + 64 * 4 + 2 * 64 * 4 + 64 * 594 * 4 + 64
+    assert gdn.accept_workspace_bytes(64, 8, 151936, False) == 64 * 8 * 16 + 64 * 4 + 2 * 64 * 4 + 64
+    call = lambda V=1024, T=8, sampled=1, tau=1.0, ws=fake, nbytes=1 << 30, draft=fake, u=fake, dtype=1: lib.gdn_accept(
+        ctypes.byref(gdn._accept_shape(4, T, V, gdn.torch.bfloat16 if dtype else gdn.torch.float32, sampled, tau)),
+        fake, draft, fake, u, fake, fake, ws, nbytes, None)
+    assert call(V=1020) == UNSUP and "multiple of 8" in lib.gdn_last_error().decode()
+    assert call(T=17) == UNSUP
+    assert call(tau=0.0) == INVALID and "temperature" in lib.gdn_last_error().decode()
+    assert call(draft=None) == INVALID and "draft_logits is NULL" in lib.gdn_last_error().decode()
+    assert call(u=None) == INVALID and "uniforms is NULL" in lib.gdn_last_error().decode()
+    assert call(sampled=0, draft=None, u=None, nbytes=16) == WORKSPACE
+    assert call(ws=fake + 8) == INVALID and "workspace not 16-byte aligned" in lib.gdn_last_error().decode()

@@ -47,7 +47,10 @@ KERNEL_SOURCES = {
     "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
     "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
     "short_conv": [_CSRC + "gdn_conv.cu"] + _HEADERS,
+    "accept": [_CSRC + "gdn_accept.cu"] + _HEADERS,
+    "accept_greedy": [_CSRC + "gdn_accept.cu"] + _HEADERS,
 }
+ACCEPT_V = 151936   # vocabulary of the acceptance workloads (the pages give none: the Qwen tokenizer's)
 CONV_K, CONV_LAYERS = 4, 48   # short convolution: filter taps; one convolution per GDN layer
 
 
@@ -180,8 +183,25 @@ def gated_bytes(w):
     return algorithmic_bytes(w) + w.B * w.T * w.H_v * w.d_v * el + w.d_v * 4
 
 
+def accept_bytes(w, sampled, V=ACCEPT_V):
+    """Bytes one acceptance call must move: every logit read once (target rows, and the draft
+    rows in sampled mode), the tokens, the uniforms and the two outputs."""
+    el = 2 if w.in_dtype == "bf16" else 4
+    n = w.B * w.T * V * el + (w.B * (w.T - 1) * V * el if sampled else 0)
+    return n + w.B * w.T * 4 + (w.B * w.T * 4 if sampled else 0) + 2 * w.B * 4
+
+
 def workload_config(name):
     """The JSON `config` of a workload (what it is, with its sizes)."""
+    if name in ("accept", "accept_greedy"):
+        w = workload("batched_verify")
+        sampled = name == "accept"
+        return {"workload": name, "B": w.B, "T": w.T, "V": ACCEPT_V, "logits": "bf16",
+                "mode": "exact speculative sampling, temperature 1" if sampled else "greedy",
+                "inputs": "target logits N(0,1) [B,T,V]" + (", draft logits target + N(0,0.5) [B,T-1,V], uniforms"
+                                                             if sampled else "") +
+                          "; 80% of drafted tokens planted with +8 in both models",
+                "l2": "inputs larger than L2 (%.0f MB moved per step, L2 126 MB)" % (accept_bytes(w, sampled) / 1e6)}
     if name == "verify_gated":
         c = workload_config("batched_verify")
         w = workload("batched_verify")
@@ -392,6 +412,41 @@ class ShortConv:
         return workload_config("short_conv")
 
 
+class Accept:
+    """accept / accept_greedy: device-side acceptance of a batch of verify blocks (B = 64, T = 8,
+    V = 151,936 bf16 logits): one C-ABI call per step (two kernels)."""
+
+    def __init__(self, name, rank, dev):
+        from gated_deltanet_mixer_verify_b200 import gdn
+        from gated_deltanet_mixer_verify_b200.inputs import make_accept_inputs
+        self.gdn = gdn
+        self.name = name
+        self.sampled = name == "accept"
+        self.w = workload("batched_verify", seed=rank_seed(workload("batched_verify").seed, rank))
+        self.host = make_accept_inputs(self.w, V=ACCEPT_V)
+        self.x = {k: v.to(dev) for k, v in self.host.items()}
+        B, T = self.w.B, self.w.T
+        self.ws = torch.empty(gdn.accept_workspace_bytes(B, T, ACCEPT_V, self.sampled), dtype=torch.uint8, device=dev)
+        self.L = torch.empty(B, dtype=torch.int32, device=dev)
+        self.o = torch.empty(B, dtype=torch.int32, device=dev)   # the next tokens
+        self.launches_per_step = 2 if self.sampled else 1
+        self.calls_per_step = 1
+        self.bytes = accept_bytes(self.w, self.sampled)
+        self.units = B * T
+
+    def step(self, x=None):
+        x = x or self.x
+        self.gdn.accept(x["target"], x["tokens"], x["draft"] if self.sampled else None,
+                        x["uniforms"] if self.sampled else None, workspace=self.ws, accept_len=self.L,
+                        next_token=self.o)
+
+    def per_step_inputs(self):
+        return ["target", "tokens"] + (["draft", "uniforms"] if self.sampled else [])
+
+    def config(self):
+        return workload_config(self.name)
+
+
 class SingleSeq:
     """single_seq_verify: one sequence through 48 distinct layers, one launch per layer,
     captured once as a CUDA graph; a step replays the graph."""
@@ -486,7 +541,7 @@ class Prefill:
 
 WORKLOADS = {"batched_verify": Verify, "decode": Verify, "single_seq_verify": SingleSeq,
              "prefill": Prefill, "commit_next_verify": CommitNext, "short_conv": ShortConv,
-             "verify_gated": VerifyGated}
+             "verify_gated": VerifyGated, "accept": Accept, "accept_greedy": Accept}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -496,9 +551,28 @@ def oracle_sample(name, budget_s, rank=0):
     Returns (seconds per unit, units timed, description, threads)."""
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    shape = "batched_verify" if name in ("commit_next_verify", "short_conv", "verify_gated") else name
+    shape = "batched_verify" if name in ("commit_next_verify", "short_conv", "verify_gated", "accept",
+                                         "accept_greedy") else name
     w = workload(shape, seed=rank_seed(workload(shape).seed, rank))
     threads = orc.max_threads()
+    if name in ("accept", "accept_greedy"):
+        from gated_deltanet_mixer_verify_b200.inputs import make_accept_inputs
+        sampled = name == "accept"
+        n_seq = 4
+        x = make_accept_inputs(workload(shape, B=n_seq), V=ACCEPT_V)
+        f = {k: v.double().numpy() for k, v in x.items() if k != "tokens"}
+        reps, t_total = 0, 0.0
+        while t_total < budget_s or reps == 0:
+            t0 = time.perf_counter()
+            orc.accept(f["target"], x["tokens"].numpy(), f["draft"] if sampled else None,
+                       f["uniforms"] if sampled else None, sampled=sampled)
+            t_total += time.perf_counter() - t0
+            reps += 1
+            if reps >= 1000:
+                break
+        desc = "%d sequences x T=%d x V=%d, %s, %d repetition(s)" % (n_seq, w.T, ACCEPT_V,
+                                                                     "sampled" if sampled else "greedy", reps)
+        return t_total / (reps * n_seq), n_seq * reps, desc, 1
     if name == "short_conv":
         from gated_deltanet_mixer_verify_b200.inputs import make_conv_block
         n_seq = 16
@@ -555,7 +629,9 @@ def cpu_value(name, per_unit_s):
     """The workload metric (GB/s or tok/s) the oracle reaches at per_unit_s per unit."""
     if name == "prefill":
         return 1.0 / per_unit_s, "tok/s"
-    if name == "short_conv":
+    if name in ("accept", "accept_greedy"):
+        per_seq_bytes = accept_bytes(workload("batched_verify", B=1), name == "accept")
+    elif name == "short_conv":
         per_seq_bytes = conv_bytes(workload("batched_verify", B=1))
     elif name == "verify_gated":
         per_seq_bytes = gated_bytes(workload("batched_verify", B=1))
@@ -584,6 +660,16 @@ def run_reference(args, rank, world):
                                   f["dt_bias"], None)
         units_per_step = 256 * 3 / workload(name).H_v          # prompt tokens (all heads)
         desc = "256 tokens x 3 of 48 value heads per step (fp64 recurrence)"
+    elif name in ("accept", "accept_greedy"):
+        from gated_deltanet_mixer_verify_b200.inputs import make_accept_inputs
+        sampled = name == "accept"
+        sub = workload("batched_verify", B=2)
+        xa = make_accept_inputs(sub, V=ACCEPT_V)
+        fa = {k: v.double().numpy() for k, v in xa.items() if k != "tokens"}
+        run = lambda: orc.accept(fa["target"], xa["tokens"].numpy(), fa["draft"] if sampled else None,
+                                 fa["uniforms"] if sampled else None, sampled=sampled)
+        units_per_step = accept_bytes(sub, sampled) / 1e9
+        desc = "2 sequences x T=8 x V=%d per step, %s" % (ACCEPT_V, "sampled" if sampled else "greedy")
     elif name == "short_conv":
         from gated_deltanet_mixer_verify_b200.inputs import make_conv_block
         sub = workload("batched_verify", B=4)
@@ -627,7 +713,7 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference", "config": workload_config(name),
             "cpu_baseline": {"value": value, "unit": unit,
-                             "cores": 1 if name == "short_conv" else orc.max_threads(),
+                             "cores": 1 if name in ("short_conv", "accept", "accept_greedy") else orc.max_threads(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -706,7 +792,7 @@ def main():
     e2e = None
     if hasattr(wl, "e2e"):
         e2e = wl.e2e(args.steps, barrier, world, dev)
-    elif isinstance(wl, (Verify, Prefill)):
+    elif isinstance(wl, (Verify, Prefill, Accept)):
         names = wl.per_step_inputs()
         host = {k: wl.host[k].pin_memory() for k in names}
         dev_in = dict(wl.x)
@@ -759,8 +845,9 @@ def main():
         else:
             value = weak_scaling_throughput(wl.bytes, world, ms_per_step / 1e3) / 1e9
             unit = "GB/s"
-            kernel_ms = statistics.mean(step_ms) / wl.launches_per_step
-            per_launch_bytes = wl.bytes / wl.launches_per_step
+            calls = getattr(wl, "calls_per_step", wl.launches_per_step)   # acceptance: one call, two kernels
+            kernel_ms = statistics.mean(step_ms) / calls
+            per_launch_bytes = wl.bytes / calls
             achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
             roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                         "frac": achieved / hbm_peak, "peak_source": "%s hbm_gbs (%s)" % (src, peak_kind),

@@ -568,8 +568,8 @@ static gdn_status check_accept(const gdn_accept_shape* s, const char* who) {
     if (s->B < 0 || s->T < 1 || s->V < 1)
         return fail(GDN_ERR_INVALID_ARG, "%s: sizes must be positive (B may be 0)", who);
     if (s->T > 16) return fail(GDN_ERR_UNSUPPORTED, "%s: T %d > 16", who, s->T);
-    if (s->V % 8 != 0 || s->V > (1 << 24))
-        return fail(GDN_ERR_UNSUPPORTED, "%s: V must be a multiple of 8 up to 2^24 (got %d)", who, s->V);
+    if (s->V % 8 != 0 || s->V > (1 << 18))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: V must be a multiple of 8 up to 2^18 (got %d)", who, s->V);
     if (s->B > (1 << 20)) return fail(GDN_ERR_UNSUPPORTED, "%s: B > 2^20", who);
     if (s->logits_dtype != GDN_F32 && s->logits_dtype != GDN_BF16)
         return fail(GDN_ERR_INVALID_ARG, "%s: logits_dtype %d unknown", who, s->logits_dtype);

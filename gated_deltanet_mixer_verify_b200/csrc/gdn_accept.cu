@@ -76,34 +76,44 @@ __device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2)
     m = mn;
 }
 
-// p_t(d) and q_t(d) from the statistics; the acceptance decisions and n of sequence b.
+// The decisions of sequence b, one draft per lane (warp-wide call): greedy compares the draft
+// with the row's first argmax; sampled tests u * q < p with p, q from the row statistics. n is
+// the length of the leading run of survivors; lane 0 writes accept_len = n + 1 (and the greedy
+// next token) and keeps n for the draw.
 template <typename LT>
-__device__ int leading_run(const AcceptArgs& a, const RowStat* st, int b) {
-    const LT* tg = static_cast<const LT*>(a.target);
-    const LT* dr = static_cast<const LT*>(a.draft);
-    const float c = kLog2e / a.tau;
-    int n = 0;
-    for (int t = 0; t + 1 < a.T; ++t) {
+__device__ void decide(const AcceptArgs& a, int b, int lane) {
+    bool ok = false;
+    const int t = lane;
+    if (t + 1 < a.T) {
         const int d = a.tokens[(int64_t)b * a.T + t + 1];
-        bool ok;
+        const RowStat* st = a.stats;
         if (!a.sampled) {
             ok = d == __ldcg(&st[(int64_t)b * a.T + t].arg);
-        } else if (d < 0 || d >= a.V) {
-            ok = false;
-        } else {
-            const RowStat sp = {__ldcg(&st[(int64_t)b * a.T + t].m), __ldcg(&st[(int64_t)b * a.T + t].s), 0, 0};
+        } else if (d >= 0 && d < a.V) {
+            const float c = kLog2e / a.tau;
+            const int64_t pr = (int64_t)b * a.T + t;
             const int64_t qr = (int64_t)a.B * a.T + (int64_t)b * (a.T - 1) + t;
-            const RowStat sq = {__ldcg(&st[qr].m), __ldcg(&st[qr].s), 0, 0};
-            const float p = exp2_approx(ld1l(tg, ((int64_t)b * a.T + t) * a.V + d) * c - sp.m) / sp.s;
-            const float q = exp2_approx(ld1l(dr, ((int64_t)b * (a.T - 1) + t) * a.V + d) * c - sq.m) / sq.s;
+            const float lp = ld1l(static_cast<const LT*>(a.target), pr * a.V + d);
+            const float lq = ld1l(static_cast<const LT*>(a.draft), ((int64_t)b * (a.T - 1) + t) * a.V + d);
+            const float p = exp2_approx(lp * c - __ldcg(&st[pr].m)) / __ldcg(&st[pr].s);
+            const float q = exp2_approx(lq * c - __ldcg(&st[qr].m)) / __ldcg(&st[qr].s);
             ok = a.u[(int64_t)b * a.T + t + 1] * q < p;
         }
-        if (!ok) break;
-        ++n;
     }
-    return n;
+    const unsigned bits = __ballot_sync(kFull, ok);
+    const unsigned full = (a.T - 1 >= 32) ? kFull : ((1u << (a.T - 1)) - 1u);
+    const int n = ((bits & full) == full) ? a.T - 1 : __ffs(~bits) - 1;
+    if (lane == 0) {
+        a.accept_len[b] = n + 1;
+        a.nsurv[b] = n;
+        if (!a.sampled) a.next_token[b] = __ldcg(&a.stats[(int64_t)b * a.T + n].arg);
+    }
 }
 
+// One CTA per logit row (target rows, then draft rows): the row streamed once, four 8-logit
+// groups per thread in flight (addresses clamped into the row, values past its end masked, so
+// that no branch sits between the loads). The last row of a sequence (fence, then an atomic
+// counter: nothing waits) has warp 0 decide.
 template <typename LT>
 __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const AcceptArgs a) {
     const int64_t r = blockIdx.x;
@@ -115,22 +125,14 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
     const float c = kLog2e / a.tau;
     float m = -INFINITY, s = 0.f;
     int arg = 0x7fffffff;
-    // Four 8-logit groups in flight per thread.
     for (int base = 8 * tid; base < a.V; base += 4 * 8 * kRowThreads) {
         float x[4][8];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const int i = base + g * 8 * kRowThreads;
-            if (i < a.V) {
-                ld8l<LT>(row + i, x[g]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[g][e] = -INFINITY;
-            }
-        }
+        for (int g = 0; g < 4; ++g) ld8l<LT>(row + min(base + g * 8 * kRowThreads, a.V - 8), x[g]);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const int i = base + g * 8 * kRowThreads;
+            if (i >= a.V) continue;
             if (!a.sampled) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
@@ -139,15 +141,17 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
                         arg = i + e;
                     }
             } else {
-                float lm = -INFINITY;
+                // one exponential per logit: the running sum is rescaled only when the running
+                // maximum grows (rarely, after a thread's first groups)
+                float lm = m;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[g][e] * c);
-                if (lm > -INFINITY) {
-                    float ls = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ls += exp2_approx(x[g][e] * c - lm);
-                    merge_ms(m, s, lm, ls);
+                if (lm > m) {
+                    s *= exp2_approx(m - lm);   // 0 when m is still -inf
+                    m = lm;
                 }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s += exp2_approx(x[g][e] * c - m);
             }
         }
     }
@@ -182,33 +186,39 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
         last = atomicAdd(&a.counters[b], 1) == rows_per_seq - 1;
     }
     __syncthreads();
-    if (!last || tid != 0) return;
-    // The last row of sequence b: every row's statistics are in place.
+    if (!last || warp != 0) return;
     __threadfence();
-    const int n = leading_run<LT>(a, a.stats, b);
-    a.accept_len[b] = n + 1;
-    a.nsurv[b] = n;
-    if (!a.sampled) a.next_token[b] = __ldcg(&a.stats[(int64_t)b * a.T + n].arg);
+    decide<LT>(a, b, lane);
 }
 
-// Residual (or target) weight of logit j of sequence b's row n, from the statistics.
+// Logits j .. j+7 of the target row (and the draft row) as raw values.
 template <typename LT>
-__device__ __forceinline__ void weights8(const AcceptArgs& a, const LT* pr, const LT* qr, int j, float pm, float ps,
-                                         float qm, float qs, float (&w)[8]) {
-    const float c = kLog2e / a.tau;
-    float x[8];
-    ld8l<LT>(pr + j, x);
+__device__ __forceinline__ void load_pair(const LT* pr, const LT* qr, int j, int V, float (&x)[8], float (&y)[8]) {
+    if (j < V) {
+        ld8l<LT>(pr + j, x);
+        if (qr) ld8l<LT>(qr + j, y);
+    } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = exp2_approx(x[e] * c - pm) / ps;
-    if (qr) {
-        float y[8];
-        ld8l<LT>(qr + j, y);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = fmaxf(w[e] - exp2_approx(y[e] * c - qm) / qs, 0.f);
+        for (int e = 0; e < 8; ++e) x[e] = y[e] = -INFINITY;
     }
 }
 
-// grid (B, kSplit): tile sums of row n's residual; the last CTA of the sequence draws.
+// Residual (or target) weights from raw logits and the row statistics (pi, qi: the reciprocals
+// of the row sums).
+__device__ __forceinline__ void weights_of(const float (&x)[8], const float (&y)[8], bool resid, float c, float pm,
+                                           float pi, float qm, float qi, float (&w)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        float v = exp2_approx(x[e] * c - pm) * pi;
+        if (resid) v = fmaxf(v - exp2_approx(y[e] * c - qm) * qi, 0.f);
+        w[e] = x[e] == -INFINITY ? 0.f : v;
+    }
+}
+
+constexpr int kMaxTiles = 1024;   // V <= 2^18
+
+// grid (B, kSplit): tile sums of row n's residual, 4 tiles in flight per warp; the last CTA of
+// the sequence stages all tile sums in shared memory and draws the token by inverse CDF.
 template <typename LT>
 __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const AcceptArgs a) {
     const int b = blockIdx.x;
@@ -224,98 +234,108 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
         qm = __ldcg(&a.stats[q].m);
         qs = __ldcg(&a.stats[q].s);
     }
-    const float pm = __ldcg(&a.stats[prow].m), ps = __ldcg(&a.stats[prow].s);
+    const bool resid = qr != nullptr;
+    const float pm = __ldcg(&a.stats[prow].m), pi = 1.f / __ldcg(&a.stats[prow].s);
+    qs = 1.f / qs;   // from here on the reciprocal
+    const float c = kLog2e / a.tau;
     const int ntiles = (a.V + kTile - 1) / kTile;
     float* tsum = a.tiles + (int64_t)b * ntiles;
-    // Tiles blockIdx.y, +kSplit, ... ; a warp per tile, 8 logits per lane.
-    for (int tile = blockIdx.y + kSplit * warp; tile < ntiles; tile += kSplit * (kSplitThreads / 32)) {
-        const int j = tile * kTile + 8 * lane;
-        float acc = 0.f;
-        if (j < a.V) {
+    constexpr int kStride = kSplit * (kSplitThreads / 32);   // tiles between a warp's iterations
+    for (int t0 = blockIdx.y + kSplit * warp; t0 < ntiles; t0 += 4 * kStride) {
+        float x[4][8], y[4][8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) load_pair<LT>(pr, qr, (t0 + k * kStride) * kTile + 8 * lane, a.V, x[k], y[k]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int tile = t0 + k * kStride;
             float w[8];
-            weights8<LT>(a, pr, qr, j, pm, ps, qm, qs, w);
+            weights_of(x[k], y[k], resid, c, pm, pi, qm, qs, w);
+            float acc = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc += w[e];
+            acc = warp_sum(acc);
+            if (lane == 0 && tile < ntiles) tsum[tile] = acc;
         }
-        acc = warp_sum(acc);
-        if (lane == 0) tsum[tile] = acc;
     }
     __shared__ bool last;
+    __shared__ float sts[kMaxTiles];
     __syncthreads();
     if (tid == 0) {
         __threadfence();
         last = atomicAdd(&a.counters[a.B + b], 1) == kSplit - 1;
     }
     __syncthreads();
-    if (!last || warp != 0) return;
+    if (!last) return;
     __threadfence();
-    // Warp 0 of the last CTA: the total and the tile holding u_0 * total (lane L covers a
-    // contiguous range of tiles), then the logit inside that tile.
+    for (int t = tid; t < ntiles; t += kSplitThreads) sts[t] = __ldcg(&tsum[t]);
+    __syncthreads();
+    if (warp != 0) return;
+    // Warp 0: the total and the tile holding u_0 * total (lane L sums a contiguous range of
+    // tiles), then the logit inside that tile.
     const int per = (ntiles + 31) / 32;
-    const int t0 = lane * per, t1 = min(t0 + per, ntiles);
+    const int r0 = min(lane * per, ntiles), r1 = min(r0 + per, ntiles);
     float mine = 0.f;
-    for (int t = t0; t < t1; ++t) mine += __ldcg(&tsum[t]);
+    for (int t = r0; t < r1; ++t) mine += sts[t];
     float incl = mine;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += y;
+        const float v = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += v;
     }
     const float total = __shfl_sync(kFull, incl, 31);
     const float target = a.u[(int64_t)b * a.T] * total;
     const unsigned hit = __ballot_sync(kFull, incl > target && mine > 0.f);
-    const bool fallback = hit == 0;   // warp-uniform
+    const bool fallback = hit == 0;   // rounding put u_0 * total at the very end
     int tile = -1;
     float before = 0.f;
     if (!fallback) {
         const int L = __ffs(hit) - 1;
         if (lane == L) {
             float cum = incl - mine;
-            for (int t = t0; t < t1; ++t) {
-                const float v = __ldcg(&tsum[t]);
-                if (cum + v > target && v > 0.f) {
+            for (int t = r0; t < r1; ++t) {
+                if (cum + sts[t] > target && sts[t] > 0.f) {
                     tile = t;
                     break;
                 }
-                cum += v;
+                cum += sts[t];
             }
-            if (tile < 0) {   // rounding: the last positive tile of the range
-                for (int t = t1 - 1; t >= t0; --t)
-                    if (__ldcg(&tsum[t]) > 0.f) {
+            if (tile < 0)
+                for (int t = r1 - 1; t >= r0; --t)
+                    if (sts[t] > 0.f) {
                         tile = t;
                         break;
                     }
-            }
             before = cum;
         }
         tile = __shfl_sync(kFull, tile, L);
         before = __shfl_sync(kFull, before, L);
-    } else {   // rounding at the very end: the last tile with mass
+    } else {
         int lt = -1;
         for (int t = ntiles - 1 - lane; t >= 0; t -= 32)
-            if (__ldcg(&tsum[t]) > 0.f) {
+            if (sts[t] > 0.f) {
                 lt = t;
                 break;
             }
-        tile = __reduce_max_sync(kFull, lt);   // its last positive logit is taken below
+        tile = __reduce_max_sync(kFull, lt);
     }
     if (tile < 0) {
         if (lane == 0) a.next_token[b] = 0;
         return;
     }
     const int j = tile * kTile + 8 * lane;
-    float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (j < a.V) weights8<LT>(a, pr, qr, j, pm, ps, qm, qs, w);
+    float x[8], y[8], w[8];
+    load_pair<LT>(pr, qr, j, a.V, x, y);
+    weights_of(x, y, resid, c, pm, pi, qm, qs, w);
     float mine2 = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) mine2 += w[e];
     float incl2 = mine2;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(kFull, incl2, off);
-        if (lane >= off) incl2 += y;
+        const float v = __shfl_up_sync(kFull, incl2, off);
+        if (lane >= off) incl2 += v;
     }
-    // The first logit whose running mass passes the target; otherwise the tile's last positive.
+    // The first logit whose running mass passes the target; else the tile's last positive one.
     int found = 0x7fffffff, lastpos = -1;
     float cum = before + incl2 - mine2;
 #pragma unroll
@@ -336,20 +356,21 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled) {
     const size_t rows = (size_t)B * T + (sampled ? (size_t)B * (T - 1) : 0);
     const size_t ntiles = ((size_t)V + kTile - 1) / kTile;
-    return rows * sizeof(RowStat) + (size_t)B * 4 /* nsurv */ + (size_t)2 * B * 4 /* counters */ +
+    return rows * sizeof(RowStat) /* stats */ + (size_t)2 * B * 4 /* counters */ + (size_t)B * 4 /* n */ +
            (sampled ? (size_t)B * ntiles * 4 : 0) + 64;
 }
 
 cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream) {
-    // Workspace: statistics, then n per sequence, the counters, the tile sums.
-    unsigned char* w = static_cast<unsigned char*>(workspace);
+    // Workspace: row statistics, the counters (rows done per sequence, draw CTAs done per
+    // sequence), n per sequence, the tile sums.
     const size_t rows = (size_t)a.B * a.T + (a.sampled ? (size_t)a.B * (a.T - 1) : 0);
+    unsigned char* w = static_cast<unsigned char*>(workspace);
     a.stats = reinterpret_cast<RowStat*>(w);
     w += rows * sizeof(RowStat);
-    a.nsurv = reinterpret_cast<int*>(w);
-    w += (size_t)a.B * 4;
     a.counters = reinterpret_cast<int*>(w);
     w += (size_t)2 * a.B * 4;
+    a.nsurv = reinterpret_cast<int*>(w);
+    w += (size_t)a.B * 4;
     a.tiles = reinterpret_cast<float*>(w);
     cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)2 * a.B * 4, stream);
     if (e != cudaSuccess) return e;
@@ -357,9 +378,9 @@ cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream) {
     else gdn_accept_rows_kernel<float><<<(unsigned)rows, kRowThreads, 0, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || !a.sampled) return e;
-    const dim3 grid(a.B, kSplit);
-    if (a.bf16) gdn_accept_draw_kernel<__nv_bfloat16><<<grid, kSplitThreads, 0, stream>>>(a);
-    else gdn_accept_draw_kernel<float><<<grid, kSplitThreads, 0, stream>>>(a);
+    const dim3 dgrid(a.B, kSplit);
+    if (a.bf16) gdn_accept_draw_kernel<__nv_bfloat16><<<dgrid, kSplitThreads, 0, stream>>>(a);
+    else gdn_accept_draw_kernel<float><<<dgrid, kSplitThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -112,10 +112,10 @@ struct AcceptArgs {
     int32_t* accept_len;         // [B] out
     int32_t* next_token;         // [B] out
     int32_t* status_word;
-    AcceptRowStat* stats;        // set by the launcher from the workspace
-    int* nsurv;
-    int* counters;
-    float* tiles;
+    AcceptRowStat* stats;        // set by the launcher from the workspace: row statistics,
+    int* nsurv;                  // surviving drafts per sequence,
+    int* counters;               // [2 B]: rows done per sequence, draw CTAs done per sequence,
+    float* tiles;                // residual tile sums per sequence
 };
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled);
 cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream);

@@ -338,7 +338,7 @@ gdn_status gdn_short_conv(const gdn_shape* shape, int32_t conv_k,
  * draft t+1 iff it is the first index of the maximum of target row t; sampled keeps it iff
  * uniforms[b][t+1] * q_t(d) < p_t(d). Decisions are taken in fp32. A draw takes the first index
  * whose running mass exceeds u times the total. workspace: gdn_accept_workspace_bytes, 16-byte
- * aligned, contents irrelevant (the call zeroes what it needs). V a multiple of 8, up to 2^24;
+ * aligned, contents irrelevant (the call zeroes what it needs). V a multiple of 8, up to 2^18;
  * T 1..16.
  */
 typedef struct {

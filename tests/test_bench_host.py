@@ -77,3 +77,18 @@ def test_gated_bytes_and_reference_arm(bench):
     assert out.returncode == 0, out.stderr[-2000:]
     d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
     assert d["config"]["workload"] == "verify_gated" and d["value"] > 0
+
+
+@pytest.mark.parametrize("name", ["accept", "accept_greedy"])
+def test_accept_bytes_and_reference_arm(bench, name):
+    w = workload("batched_verify")
+    V = 151936
+    sampled = name == "accept"
+    expect = 64 * 8 * V * 2 + (64 * 7 * V * 2 if sampled else 0) + 64 * 8 * 4 + (64 * 8 * 4 if sampled else 0) + 2 * 64 * 4
+    assert bench.accept_bytes(w, sampled) == expect
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", name, "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"]["workload"] == name and d["value"] > 0 and d["cpu_baseline"]["cores"] == 1

@@ -620,6 +620,14 @@ gdn_status gdn_accept(const gdn_accept_shape* shape, const void* target_logits, 
     return launched(gdn::launch_accept(a, workspace, static_cast<cudaStream_t>(stream)), who);
 }
 
+gdn_status gdn_selftest_bounded_wait(int32_t* status_word, uint32_t polls, void* stream) {
+    const char* who = "gdn_selftest_bounded_wait";
+    if (!status_word || (reinterpret_cast<uintptr_t>(status_word) & 3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: status_word is NULL or misaligned", who);
+    if (polls == 0 || polls > (1u << 20)) return fail(GDN_ERR_INVALID_ARG, "%s: polls must be 1..2^20", who);
+    return launched(gdn::launch_bounded_wait_selftest(status_word, polls, static_cast<cudaStream_t>(stream)), who);
+}
+
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
 
 }  // extern "C"

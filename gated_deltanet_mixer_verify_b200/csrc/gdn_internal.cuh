@@ -118,6 +118,9 @@ struct AcceptArgs {
     float* tiles;                // residual tile sums per sequence
 };
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled);
+
+// A bounded wait that nothing completes (gdn_selftest.cu).
+cudaError_t launch_bounded_wait_selftest(int32_t* status_word, uint32_t polls, cudaStream_t stream);
 cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.

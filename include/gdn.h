@@ -363,6 +363,14 @@ size_t gdn_stash_bytes(const gdn_shape* shape);
  * value head. */
 size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk);
 
+/*
+ * gdn_selftest_bounded_wait -- test hook for the failure path that every bounded wait in the
+ * library shares: one kernel waits, with the same helper, on an mbarrier that nothing completes;
+ * after `polls` polls (1..2^20) it gives up, ORs GDN_STATUS_WAIT_TIMEOUT into *status_word
+ * (device int32) and returns. The context stays usable. Nothing faults, traps or hangs.
+ */
+gdn_status gdn_selftest_bounded_wait(int32_t* status_word, uint32_t polls, void* stream);
+
 /* Static description of a status code. */
 const char* gdn_status_string(gdn_status status);
 

@@ -215,3 +215,11 @@ def test_accept_validates_on_the_host(gdn):
     assert call(u=None) == INVALID and "uniforms is NULL" in lib.gdn_last_error().decode()
     assert call(sampled=0, draft=None, u=None, nbytes=16) == WORKSPACE
     assert call(ws=fake + 8) == INVALID and "workspace not 16-byte aligned" in lib.gdn_last_error().decode()
+
+
+def test_selftest_bounded_wait_validates_on_the_host(gdn):
+    lib = gdn.lib()
+    assert lib.gdn_selftest_bounded_wait(None, 16, None) == -1
+    assert lib.gdn_selftest_bounded_wait(0x100002, 16, None) == -1          # misaligned
+    assert lib.gdn_selftest_bounded_wait(0x100000, 0, None) == -1
+    assert lib.gdn_selftest_bounded_wait(0x100000, (1 << 20) + 1, None) == -1

@@ -1,0 +1,31 @@
+"""The failure path of the bounded waits, on the GPU, without a fault: a wait on an mbarrier
+that nothing completes gives up after its poll limit, reports the wait-timeout bit in the
+status word and returns; the context stays usable (a verify call after it is still exact)."""
+import pytest
+import torch
+
+from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload
+from gdn_helpers import TOL, gpu_verify, oracle_verify, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gdn(cuda_device):
+    from gated_deltanet_mixer_verify_b200 import build, gdn as g
+    build.build()
+    return g
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(gdn):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gdn.selftest_bounded_wait(status, polls=1024)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 2
+    # the context still computes: a verify call afterwards matches the oracle
+    w = workload("batched_verify", B=2, seed=95)
+    x = make_inputs(w)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, S = gpu_verify(gdn, to_dev(x), x["accept_len"].numpy(), status=st2)
+    o_ref, S_ref, _ = oracle_verify(x, x["accept_len"].numpy())
+    assert rel_err(o, o_ref) <= TOL and rel_err(S, S_ref) <= TOL and int(st2.item()) == 0

@@ -793,25 +793,54 @@ def main():
     if hasattr(wl, "e2e"):
         e2e = wl.e2e(args.steps, barrier, world, dev)
     elif isinstance(wl, (Verify, Prefill, Accept)):
+        # Every step copies its own inputs in from pinned host memory and its result out, as a
+        # serving loop does: double-buffered, on an upload and a download stream, so that step
+        # i+1's inputs arrive and step i-1's result leaves while step i computes. Events order
+        # each buffer's reuse (inputs after the step that read them, outputs after the copy out).
         names = wl.per_step_inputs()
         host = {k: wl.host[k].pin_memory() for k in names}
-        dev_in = dict(wl.x)
-        dev_in.update({k: torch.empty_like(wl.x[k]) for k in names})
-        o_host = torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory()
+        dev_in = []
+        for _ in range(2):
+            d = dict(wl.x)
+            d.update({k: torch.empty_like(wl.x[k]) for k in names})
+            dev_in.append(d)
+        o_dev = [wl.o, torch.empty_like(wl.o)]
+        o_host = [torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory() for _ in range(2)]
         h2d = sum(host[k].numel() * host[k].element_size() for k in names)
-        d2h = o_host.numel() * o_host.element_size()
+        d2h = o_host[0].numel() * o_host[0].element_size()
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        drained = [torch.cuda.Event() for _ in range(2)]
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize(dev)
         e_start.record(stream)
-        for _ in range(args.steps):
-            for k in names:
-                dev_in[k].copy_(host[k], non_blocking=True)
-            wl.step(dev_in)
-            o_host.copy_(wl.o, non_blocking=True)
+        up.wait_event(e_start)
+        for i in range(args.steps):
+            j = i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(computed[j])       # step i-2 has read dev_in[j]
+                for k in names:
+                    dev_in[j][k].copy_(host[k], non_blocking=True)
+                copied[j].record(up)
+            stream.wait_event(copied[j])
+            if i >= 2:
+                stream.wait_event(drained[j])        # step i-2's result has left o_dev[j]
+            wl.o = o_dev[j]
+            wl.step(dev_in[j])
+            computed[j].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[j])
+                o_host[j].copy_(o_dev[j], non_blocking=True)
+                drained[j].record(down)
+        for j in range(2):
+            stream.wait_event(drained[j])
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
+        wl.o = o_dev[0]
         e_s = max_over_ranks(e_start.elapsed_time(e_end)) / args.steps / 1e3
         if isinstance(wl, Prefill):
             e2e = {"value": weak_scaling_throughput(wl.units, world, e_s), "unit": "tok/s"}

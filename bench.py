@@ -870,6 +870,18 @@ def main():
                         "traffic": ncu_traffic(args.workload), "kernel": wl.phase_kernel[k],
                         "algorithmic_flops_per_launch": wl.phase_work[k],
                         "phase_ms": dict(zip(wl.phase_names, phase_ms))}
+            # and the HBM side over the whole step: the minimum bytes (q, k, v read once, the
+            # outputs written once, the final state) against the measured copy bandwidth
+            w = wl.w
+            el = 2 if w.in_dtype == "bf16" else 4
+            min_bytes = (2 * w.B * w.T * w.H_k * w.d_k * el + w.B * w.T * w.H_v * w.d_v * el
+                         + 2 * w.B * w.T * w.H_v * el + w.B * w.T * w.H_v * w.d_v * 4
+                         + w.B * w.H_v * w.d_v * w.d_k * 4)
+            hbm_gbs = min_bytes / (ms_per_step / 1e3) / 1e9
+            roofline["hbm"] = {"achieved": hbm_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_gbs / hbm_peak,
+                               "min_bytes_per_step": min_bytes,
+                               "note": "minimum bytes; the workspace (records and key/query tiles, ~3 GB "
+                                       "written and read back per step) comes on top"}
             dtype = Prefill.dtype
         else:
             value = weak_scaling_throughput(wl.bytes, world, ms_per_step / 1e3) / 1e9

@@ -343,6 +343,18 @@ size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk) 
     return gdn::prefill_workspace_bytes(shape->B, shape->T, shape->H_k, shape->H_v, shape->d_k, shape->d_v, chunk);
 }
 
+int32_t gdn_chunk_prefill_pieces(int64_t T, int32_t chunk) {
+    gdn_shape s{};
+    s.B = 1;
+    s.T = 1;
+    s.H_k = 1;
+    s.H_v = 1;
+    s.d_k = 128;
+    s.d_v = 128;
+    if (T < 0 || gdn::check_prefill_shape(&s, chunk) != 0) return -1;
+    return gdn::prefill_pieces((long long)T);
+}
+
 // Shape, chunk and workspace checks shared by the workspace-taking prefill entry points.
 // Returns GDN_OK with *empty set when the batch is empty (nothing to launch).
 static gdn_status prefill_checks(const gdn_shape* shape, int32_t chunk, const void* workspace, size_t workspace_bytes,

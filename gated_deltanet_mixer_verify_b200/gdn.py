@@ -88,6 +88,8 @@ def _load():
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
     lib.gdn_chunk_prefill_workspace_bytes.argtypes = [S, ctypes.c_int32]
     lib.gdn_chunk_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_chunk_prefill_pieces.argtypes = [ctypes.c_int64, ctypes.c_int32]
+    lib.gdn_chunk_prefill_pieces.restype = ctypes.c_int32
     lib.gdn_status_string.argtypes = [ctypes.c_int]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error.argtypes = []
@@ -158,6 +160,12 @@ def prefill_workspace_bytes(B, T, H_k, H_v, d_k, d_v, chunk=64) -> int:
     """Bytes of workspace gdn_chunk_prefill needs for this shape."""
     return int(_load().gdn_chunk_prefill_workspace_bytes(
         ctypes.byref(make_shape(B, T, H_k, H_v, d_k, d_v)), chunk))
+
+
+def chunk_prefill_pieces(T, chunk=64) -> int:
+    """Pieces chunk_prefill splits a T-token prompt into (one preparation and one scan launch
+    each); -1 for an unsupported chunk."""
+    return int(_load().gdn_chunk_prefill_pieces(T, chunk))
 
 
 def verify_step(q, k, v, a, b, A_log, dt_bias, state_in, state_out=None, accept_len=None, o=None,

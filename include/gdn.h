@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 6   /* 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
+#define GDN_ABI_VERSION 7   /* 7: prefill in pieces; 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
 
 typedef enum {
     GDN_OK = 0,
@@ -177,6 +177,15 @@ gdn_status gdn_commit_and_verify(const gdn_shape* shape, int32_t prev_T,
  *   state_out  required; may equal state_in.
  *   workspace  device scratch of at least gdn_chunk_prefill_workspace_bytes(shape, chunk)
  *              bytes (16-byte aligned); contents on entry are ignored.
+ * Streams: a prompt of 64 chunks or more is split into gdn_chunk_prefill_pieces(T, chunk)
+ * pieces of whole chunks. The scan of piece i runs on a stream of the greatest priority that
+ * the library creates per device on first use (non-blocking), beside the preparation of piece
+ * i + 1 on `stream`; events order the pieces and join that stream back to `stream` before the
+ * call returns, so work queued on `stream` afterwards sees the finished o and state_out, and
+ * the call can be captured into a CUDA graph like any other. The first such call on a device
+ * creates the stream and its events, so make it outside stream capture. Calls from several
+ * host threads are serialised while they queue their launches, and their scans share that
+ * stream.
  */
 gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
                              const void* q, const void* k, const void* v,
@@ -186,8 +195,8 @@ gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * gdn_chunk_prefill_prepare / gdn_chunk_prefill_scan -- the two phases gdn_chunk_prefill runs
- * in order on its stream, for callers that schedule them separately (for instance the
+ * gdn_chunk_prefill_prepare / gdn_chunk_prefill_scan -- the two phases of gdn_chunk_prefill,
+ * each over the whole prompt on the given stream, for callers that schedule them separately (for instance the
  * preparation of the next prompt alongside the scan of this one, or timing each phase). Same
  * recurrence and chunk algebra as gdn_chunk_prefill; the split itself has no counterpart in
  * the source pages.
@@ -362,6 +371,11 @@ size_t gdn_stash_bytes(const gdn_shape* shape);
  * shape or chunk): per sequence and 64-token chunk, 65,536 bytes per key head and 49,728 per
  * value head. */
 size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk);
+
+/* Pieces gdn_chunk_prefill splits a T-token prompt into, each one preparation launch and one
+ * scan launch: with n = ceil(T / chunk) chunks, min(4, max(1, n / 32)) (integer division), so
+ * 1 below 64 chunks and 4 from 128; 0 for T = 0; -1 for T < 0 or an unsupported chunk. */
+int32_t gdn_chunk_prefill_pieces(int64_t T, int32_t chunk);
 
 /*
  * gdn_selftest_bounded_wait -- test hook for the failure path that every bounded wait in the

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 6
+    assert lib.gdn_abi_version() == 7
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()
@@ -122,6 +122,15 @@ def test_prefill_phase_entry_points_validate_on_the_host(gdn):
     assert "v is NULL" in lib.gdn_last_error().decode()
     empty = gdn.make_shape(B=0, T=300, H_k=2, H_v=6, d_k=128, d_v=128)
     assert lib.gdn_chunk_prefill_scan(ctypes.byref(empty), 64, *([None] * 5), 0, None) == 0
+
+
+def test_prefill_piece_rule(gdn):
+    # n = ceil(T / 64) chunks: min(4, max(1, n / 32)) pieces; 0 for an empty prompt
+    for T, want in ((0, 0), (1, 1), (2048, 1), (4032, 1), (4033, 2), (4096, 2), (6144, 3),
+                    (8128, 3), (8129, 4), (8192, 4), (8197, 4), (32768, 4), (1 << 24, 4)):
+        assert gdn.chunk_prefill_pieces(T) == want, T
+    assert gdn.chunk_prefill_pieces(-1) == -1
+    assert gdn.chunk_prefill_pieces(4096, chunk=32) == -1
 
 
 def test_commit_and_verify_validates_on_the_host(gdn):

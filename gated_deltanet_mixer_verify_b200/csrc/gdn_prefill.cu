@@ -748,9 +748,9 @@ struct PieceStreams {
     cudaEvent_t ev[kMaxPieces + 1] = {};
 };
 
-// The stream and events of the current device, created on first use; the caller holds `mu`.
-cudaError_t piece_streams(PieceStreams** out, std::mutex& mu) {
-    (void)mu;
+// The stream and events of the current device, created on first use and kept for the life of
+// the process. The caller holds launch_prefill's mutex, which guards them.
+cudaError_t piece_streams(PieceStreams** out) {
     constexpr int kMaxDevices = 64;
     static PieceStreams ps[kMaxDevices];
     int dev = 0;
@@ -854,7 +854,7 @@ cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
     PieceStreams* ps = nullptr;
-    cudaError_t e = piece_streams(&ps, mu);
+    cudaError_t e = piece_streams(&ps);
     if (e != cudaSuccess) return e;
     auto bound = [&](int i) { return (int)((long long)nch * i / np); };
     // Piece 0's preparation on the caller's stream, after the caller's earlier work.

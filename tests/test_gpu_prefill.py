@@ -150,3 +150,32 @@ def test_prefill_in_pieces_is_ordered_on_the_callers_stream(gdn):
         o_snap, s_snap = o.clone(), st.clone()
     torch.cuda.synchronize()
     assert torch.equal(o_snap, o_ref) and torch.equal(s_snap, s_ref)
+
+
+def test_prefill_in_pieces_captures_into_a_cuda_graph(gdn):
+    # The side stream joins the capture through the first event and leaves it through the
+    # last, so the 4-piece prefill replays as one graph with the eager call's bits.
+    w = workload("prefill", T=8192, H_k=2, H_v=6, seed=96, state_std=0.05)
+    xd = to_dev(make_inputs(w, gates="gentle"))
+    o_ref, s_ref = run_gpu(gdn, xd, xd["S0"])          # eager (also creates the side stream)
+    nb = gdn.prefill_workspace_bytes(w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    o = torch.zeros_like(o_ref)
+    st = torch.zeros_like(s_ref)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        gdn.chunk_prefill(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["A_log"], xd["dt_bias"], xd["S0"], st, o,
+                          workspace=ws)                 # warm on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            gdn.chunk_prefill(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["A_log"], xd["dt_bias"], xd["S0"], st,
+                              o, workspace=ws)
+    o.zero_()
+    st.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(st, s_ref)
+    del g

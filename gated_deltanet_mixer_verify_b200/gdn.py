@@ -327,7 +327,8 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, 
                   out_dtype=torch.float32, stream=None):
     """The mixer over a whole prompt: returns (o, state_out). ``state_in`` None = zero state.
     ``workspace`` (uint8 CUDA tensor) must hold prefill_workspace_bytes(); it is allocated
-    here when not given."""
+    here when not given. A prompt of 64 chunks or more runs in chunk_prefill_pieces(T) pieces,
+    the scans on a stream of the library's own, joined back to ``stream`` before it returns."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
     B, T, H_k, d_k = k.shape
     H_v, d_v = v.shape[2], v.shape[3]
@@ -353,9 +354,9 @@ def _nbytes(t: Optional[torch.Tensor]) -> int:
 def chunk_prefill_prepare(q, k, a, b, A_log, dt_bias, workspace, H_v=None, d_v=None, chunk=64,
                           l2_eps=1e-6, scale=1.0, status_word=None, out_dtype=torch.float32,
                           stream=None):
-    """First phase of chunk_prefill: the state-independent per-chunk operators of the prompt
-    into ``workspace`` (uint8 CUDA tensor of prefill_workspace_bytes()). H_v defaults to
-    a.shape[2], d_v to d_k."""
+    """First phase of chunk_prefill, over the whole prompt: the state-independent per-chunk
+    operators of the prompt into ``workspace`` (uint8 CUDA tensor of
+    prefill_workspace_bytes()). H_v defaults to a.shape[2], d_v to d_k."""
     B, T, H_k, d_k = k.shape
     H_v = a.shape[2] if H_v is None else H_v
     d_v = d_k if d_v is None else d_v
@@ -367,8 +368,9 @@ def chunk_prefill_prepare(q, k, a, b, A_log, dt_bias, workspace, H_v=None, d_v=N
 
 def chunk_prefill_scan(v, workspace, H_k, state_in=None, state_out=None, o=None, d_k=None, chunk=64,
                        status_word=None, out_dtype=torch.float32, stream=None):
-    """Second phase of chunk_prefill: the scan over the chunks of a prepared ``workspace``.
-    Returns (o, state_out); ``H_k`` (and d_k, default d_v) must match the prepare call."""
+    """Second phase of chunk_prefill, over the whole prompt: the scan over the chunks of a
+    prepared ``workspace``. Returns (o, state_out); ``H_k`` (and d_k, default d_v) must match
+    the prepare call."""
     B, T, H_v, d_v = v.shape
     d_k = d_v if d_k is None else d_k
     sh = make_shape(B, T, H_k, H_v, d_k, d_v, v.dtype, out_dtype, status_word=status_word)

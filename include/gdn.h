@@ -44,7 +44,8 @@
  *     nothing for sequence b (its state_out equals state_in) and sets bit 0
  *     (GDN_STATUS_BAD_ACCEPT) of *status_word when status_word is not NULL.
  *   - Calls that overlap on the GPU and write the same buffers race; calls on
- *     one stream are ordered.
+ *     one stream are ordered (gdn_chunk_prefill included, although a long
+ *     prompt's scans run on a stream of the library's own: see there).
  */
 #ifndef GDN_H
 #define GDN_H
@@ -56,7 +57,9 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 7   /* 7: prefill in pieces; 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
+/* 7: prefill in pieces (gdn_chunk_prefill_pieces); 6: gdn_accept; 5: gated norm;
+ * 4: gdn_short_conv; 3: commit-and-verify */
+#define GDN_ABI_VERSION 7
 
 typedef enum {
     GDN_OK = 0,

@@ -100,8 +100,9 @@ def test_prefill_batch_of_two_grouped_heads(gdn):
 
 
 def test_prefill_phases_match_the_one_call_prefill(gdn):
-    # prepare then scan (the two phases gdn_chunk_prefill runs) give the same bits; a second
-    # prompt prepared into its own workspace in between does not disturb the first.
+    # prepare then scan, each over the whole prompt, give the one-call prefill's bits (11
+    # chunks: one piece); a second prompt prepared into its own workspace in between does not
+    # disturb the first.
     w = workload("prefill", T=700, H_k=2, H_v=6, seed=80, state_std=0.05)
     x = to_dev(make_inputs(w, gates="gentle"))
     x2 = to_dev(make_inputs(workload("prefill", T=700, H_k=2, H_v=6, seed=81), gates="config"))

@@ -7,8 +7,11 @@ first use, so the input generator works on machines without the built library;
 any call into the mixer raises if the library is missing.
 """
 
-__all__ = ["verify_step", "commit", "decode_step", "chunk_prefill", "stash_bytes", "make_shape", "lib",
-           "prefill_workspace_bytes", "GdnError", "library_path"]
+__all__ = ["verify_step", "verify_step_gated", "commit", "commit_and_verify", "decode_step",
+           "short_conv", "conv_channels", "gated_rmsnorm", "accept", "accept_workspace_bytes",
+           "chunk_prefill", "chunk_prefill_prepare", "chunk_prefill_scan", "chunk_prefill_noalloc",
+           "chunk_prefill_pieces", "prefill_workspace_bytes", "stash_bytes", "selftest_bounded_wait",
+           "make_shape", "lib", "GdnError", "library_path"]
 
 
 def __getattr__(name):

@@ -232,3 +232,12 @@ def test_selftest_bounded_wait_validates_on_the_host(gdn):
     assert lib.gdn_selftest_bounded_wait(0x100002, 16, None) == -1          # misaligned
     assert lib.gdn_selftest_bounded_wait(0x100000, 0, None) == -1
     assert lib.gdn_selftest_bounded_wait(0x100000, (1 << 20) + 1, None) == -1
+
+
+def test_package_exports_every_binding_entry_point(gdn):
+    import gated_deltanet_mixer_verify_b200 as pkg
+    public = {n for n, v in vars(gdn).items()
+              if not n.startswith("_") and callable(v) and getattr(v, "__module__", None) == gdn.__name__}
+    assert public <= set(pkg.__all__), sorted(public - set(pkg.__all__))
+    for n in pkg.__all__:
+        assert getattr(pkg, n) is getattr(gdn, n), n

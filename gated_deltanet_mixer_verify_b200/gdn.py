@@ -151,6 +151,27 @@ def _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype) -> _Shape:
     return make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
 
 
+def _types(f32=(), i32=()):
+    """fp32 (states, stashes, gate parameters, weights) and int32 (counts) arguments, as
+    (name, tensor-or-None) pairs."""
+    for name, t in f32:
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32, not %s" % (name, t.dtype))
+    for name, t in i32:
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError("%s must be int32, not %s" % (name, t.dtype))
+
+
+def _dtypes(q, a, b, A_log, dt_bias, o=None, out_dtype=None, f32=(), i32=()):
+    """Element types the C ABI takes: a, b in q's dtype; A_log, dt_bias and the f32 pairs fp32;
+    the i32 pairs int32; o (when given) in out_dtype."""
+    if a.dtype != q.dtype or b.dtype != q.dtype:
+        raise TypeError("a and b must have q's dtype (%s)" % q.dtype)
+    _types((("A_log", A_log), ("dt_bias", dt_bias)) + tuple(f32), i32)
+    if o is not None and out_dtype is not None and o.dtype != out_dtype:
+        raise TypeError("o is %s but out_dtype is %s" % (o.dtype, out_dtype))
+
+
 def stash_bytes(B, T, H_k, H_v, d_k, d_v) -> int:
     """Bytes of stash a two-phase verify writes for this shape."""
     return int(_load().gdn_stash_bytes(ctypes.byref(make_shape(B, T, H_k, H_v, d_k, d_v))))
@@ -175,6 +196,8 @@ def verify_step(q, k, v, a, b, A_log, dt_bias, state_in, state_out=None, accept_
     to ``state_out`` (default: in place into ``state_in``); without it, ``stash`` (a float32
     CUDA tensor of stash_bytes()/4 elements) receives what :func:`commit` needs. Returns o."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype,
+            f32=(("state_in", state_in), ("state_out", state_out), ("stash", stash)), i32=(("accept_len", accept_len),))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     if accept_len is not None and state_out is None:
@@ -191,6 +214,7 @@ def commit(state_in, stash, accept_len, T, H_k, d_k=None, state_out=None, status
     ``T`` and ``H_k`` are the verify call's; state_out defaults to state_in (in place)."""
     B, H_v, d_v, dk = state_in.shape
     sh = make_shape(B, T, H_k, H_v, dk if d_k is None else d_k, d_v, status_word=status_word)
+    _types(f32=(("state_in", state_in), ("state_out", state_out), ("stash", stash)), i32=(("accept_len", accept_len),))
     if state_out is None:
         state_out = state_in
     _check(_load().gdn_commit(ctypes.byref(sh), _ptr(state_in), _ptr(state_out), _ptr(stash),
@@ -206,6 +230,8 @@ def commit_and_verify(q, k, v, a, b, A_log, dt_bias, state, prev_stash, prev_acc
     the state ends committed at this block's counts; without it the state ends at the
     committed previous block and ``stash`` receives this block's. Returns o."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state", state), ("prev_stash", prev_stash), ("stash", stash)),
+            i32=(("prev_accept_len", prev_accept_len), ("accept_len", accept_len)))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     _check(_load().gdn_commit_and_verify(ctypes.byref(sh), int(prev_T), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
@@ -221,6 +247,9 @@ def verify_step_gated(q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept
     """verify_step whose outputs are o / sqrt(mean(o^2) + norm_eps) * norm_w * silu(norm_z) per
     (token, value head); norm_z has v's shape and dtype, norm_w is [d_v] fp32. Returns o."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype,
+            f32=(("state_in", state_in), ("state_out", state_out), ("stash", stash), ("norm_w", norm_w)),
+            i32=(("accept_len", accept_len),))
     if norm_z.shape != v.shape or norm_z.dtype != v.dtype:
         raise ValueError("norm_z must have v's shape and dtype")
     if o is None:
@@ -314,6 +343,7 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale
                 status_word=None, out_dtype=torch.float32, stream=None):
     """One plain decoding token (T = 1): returns o and updates ``state`` in place."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state", state),))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     _check(_load().gdn_decode_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
@@ -330,6 +360,7 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, 
     here when not given. A prompt of 64 chunks or more runs in chunk_prefill_pieces(T) pieces,
     the scans on a stream of the library's own, joined back to ``stream`` before it returns."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state_in", state_in), ("state_out", state_out)))
     B, T, H_k, d_k = k.shape
     H_v, d_v = v.shape[2], v.shape[3]
     if o is None:
@@ -361,6 +392,7 @@ def chunk_prefill_prepare(q, k, a, b, A_log, dt_bias, workspace, H_v=None, d_v=N
     H_v = a.shape[2] if H_v is None else H_v
     d_v = d_k if d_v is None else d_v
     sh = make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
+    _dtypes(q, a, b, A_log, dt_bias)
     _check(_load().gdn_chunk_prefill_prepare(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(a), _ptr(b),
                                              _ptr(A_log), _ptr(dt_bias), _ptr(workspace),
                                              _nbytes(workspace), _stream(stream)))
@@ -374,6 +406,9 @@ def chunk_prefill_scan(v, workspace, H_k, state_in=None, state_out=None, o=None,
     B, T, H_v, d_v = v.shape
     d_k = d_v if d_k is None else d_k
     sh = make_shape(B, T, H_k, H_v, d_k, d_v, v.dtype, out_dtype, status_word=status_word)
+    _types(f32=(("state_in", state_in), ("state_out", state_out)))
+    if o is not None and o.dtype != out_dtype:
+        raise TypeError("o is %s but out_dtype is %s" % (o.dtype, out_dtype))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     if state_out is None:
@@ -395,6 +430,7 @@ def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, state_in=None, state_ou
     that need more raise GdnError. Calls that overlap on the GPU share that scratch and race.
     ``o`` and ``state_out`` are the caller's; they are only created here when omitted."""
     sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state_in", state_in), ("state_out", state_out)))
     B, T, H_k, d_k = k.shape
     H_v, d_v = v.shape[2], v.shape[3]
     if o is None:

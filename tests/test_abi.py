@@ -241,3 +241,28 @@ def test_package_exports_every_binding_entry_point(gdn):
     assert public <= set(pkg.__all__), sorted(public - set(pkg.__all__))
     for n in pkg.__all__:
         assert getattr(pkg, n) is getattr(gdn, n), n
+
+
+def test_binding_rejects_element_types_the_abi_does_not_take(gdn):
+    # checked before any pointer is taken or anything is launched (CPU tensors suffice here)
+    import torch
+    from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload
+    x = make_inputs(workload("batched_verify", B=2))
+    args = lambda **kw: [kw.get(n, x[n]) for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias")]
+    st = x["S0"]
+    cases = [
+        (dict(a=x["a"].float()), {}, "a and b must have q's dtype"),
+        (dict(A_log=x["A_log"].double()), {}, "A_log must be float32"),
+        ({}, dict(accept_len=x["accept_len"].long()), "accept_len must be int32"),
+        ({}, dict(state_in=st.double()), "state_in must be float32"),
+        ({}, dict(o=torch.empty(x["v"].shape, dtype=torch.bfloat16)), "o is torch.bfloat16"),
+    ]
+    for over, kw, msg in cases:
+        call = dict(state_in=st, accept_len=x["accept_len"])
+        call.update(kw)
+        with pytest.raises(TypeError, match=msg):
+            gdn.verify_step(*args(**over), call.pop("state_in"), **call)
+    with pytest.raises(TypeError, match="state must be float32"):
+        gdn.decode_step(*args(), st.half())
+    with pytest.raises(TypeError, match="state_out must be float32"):
+        gdn.chunk_prefill(*args(), None, st.double())

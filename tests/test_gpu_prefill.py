@@ -180,3 +180,15 @@ def test_prefill_in_pieces_captures_into_a_cuda_graph(gdn):
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(st, s_ref)
     del g
+
+
+def test_prefill_in_pieces_batch_of_two(gdn):
+    # two sequences (the scan's grid carries the sequence index), 65 chunks each: 2 pieces,
+    # the last chunk 4 tokens long
+    w = workload("prefill", B=2, T=4100, H_k=1, H_v=2, seed=97, state_std=0.05)
+    assert gdn.chunk_prefill_pieces(w.T) == 2
+    x = make_inputs(w, gates="gentle")
+    o_ref, S_ref = _oracle_prefill(x, True)
+    xd = to_dev(x)
+    o, S = run_gpu(gdn, xd, xd["S0"])
+    assert rel_err(o, o_ref) <= TOL_PREFILL and rel_err(S, S_ref) <= TOL_PREFILL

@@ -29,9 +29,19 @@
  *   accept_len[B] int32, on the device
  *
  * Conventions shared by every call:
- *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
- *     allocates nothing, frees nothing and keeps no device memory between calls.
- *     All tensor pointers must be 16-byte aligned.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, and all
+ *     tensor pointers must be 16-byte aligned. No call allocates or frees device
+ *     memory; scratch comes from the caller (stash, workspace arguments). The
+ *     library holds two pieces of state of its own, both for the life of the
+ *     process:
+ *       (1) a fixed device scratch array of GDN_NOALLOC_SCRATCH_BYTES (64 MiB),
+ *           part of the library's device code, so that every GPU which loads the
+ *           library holds it; only gdn_chunk_prefill_noalloc uses it;
+ *       (2) per device, one non-blocking stream of the greatest priority and a
+ *           few events, created on the first gdn_chunk_prefill (or _noalloc) of
+ *           64 chunks or more on that device; the prompt's scans run there
+ *           (see gdn_chunk_prefill).
+ *     Every other call keeps nothing between calls.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *     is the legacy default stream). No call synchronises the host, and no call
  *     copies accept_len (or anything else) to the host.

@@ -1,7 +1,7 @@
 """Benchmark of the Gated DeltaNet verify mixer on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload batched_verify|decode|single_seq_verify|prefill]
+                    [--workload all|batched_verify|decode|single_seq_verify|prefill|...]
 
 A step is one pass of the mixer over one batch of synthetic input, through the C ABI:
   batched_verify     (default) 64 sequences x 48 value heads, a 7 + 1 verify block, the
@@ -9,6 +9,10 @@ A step is one pass of the mixer over one batch of synthetic input, through the C
   decode             256 sequences, one token each, state updated in place
   single_seq_verify  one sequence through 48 distinct layers, replayed as a CUDA graph
   prefill            one 32768-token prompt, chunk 64
+The default (`all`) prints batched_verify as the headline line and nests one record per other
+workload under "configs" (decode, prefill, single_seq_verify, then commit_next_verify,
+verify_gated, short_conv, accept, accept_greedy), each with its own step time, roofline,
+clocks, e2e leg and CPU-oracle sample; `--workload NAME` prints that workload alone.
 Under torchrun each rank runs its own batch (weak scaling, no data-path collective); the
 step time is the max over ranks. `--impl reference` times the fp64 CPU oracle instead, on
 a bounded sample of the same workload, on rank 0 only.
@@ -449,19 +453,27 @@ class Accept:
 
 class SingleSeq:
     """single_seq_verify: one sequence through 48 distinct layers, one launch per layer,
-    captured once as a CUDA graph; a step replays the graph."""
+    captured once as a CUDA graph; a step replays the graph. Each input kind of all layers
+    lives in one device buffer (layer l reads slice l), and the round's one accept count in
+    one int32, so that a round's inputs arrive in one copy per kind."""
+
+    KINDS = ("q", "k", "v", "a", "b")
 
     def __init__(self, name, rank, dev):
         from gated_deltanet_mixer_verify_b200 import gdn
         self.gdn = gdn
         self.w = workload(name, seed=rank_seed(workload(name).seed, rank))
         L0 = make_inputs(self.w, layer=0)["accept_len"]
+        xs = [make_inputs(self.w, layer=l, accept_len=L0.numpy()) for l in range(self.w.layers)]
+        self.host = {k: torch.stack([x[k] for x in xs]) for k in self.KINDS}
+        self.host["accept_len"] = L0.clone()
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        self.o_all = torch.empty((self.w.layers,) + tuple(xs[0]["v"].shape), dtype=torch.float32, device=dev)
         self.layers = []
-        for l in range(self.w.layers):
-            x = make_inputs(self.w, layer=l, accept_len=L0.numpy())
-            xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-            xd["state"] = xd["S0"].clone()
-            xd["o"] = torch.empty(xd["v"].shape, dtype=torch.float32, device=dev)
+        for l, x in enumerate(xs):
+            xd = {k: self.dev[k][l] for k in self.KINDS}
+            xd.update(A_log=x["A_log"].to(dev), dt_bias=x["dt_bias"].to(dev), state=x["S0"].to(dev),
+                      accept_len=self.dev["accept_len"], o=self.o_all[l])
             self.layers.append(xd)
         self.launches_per_step = self.w.layers
         self.bytes = algorithmic_bytes(self.w) * self.w.layers
@@ -484,6 +496,32 @@ class SingleSeq:
             with torch.cuda.graph(self.graph, stream=self.stream):
                 self._eager()
         self.graph.replay()
+
+    def e2e(self, steps, barrier, world, dev):
+        """Through the public calls with host buffers: per round, every layer's q, k, v, a, b and
+        the round's accept count copied in from pinned memory (one copy per kind), the 48
+        launches (the graph), every layer's o copied out (one copy)."""
+        self.step()
+        host = {k: v.pin_memory() for k, v in self.host.items()}
+        o_host = torch.empty(self.o_all.shape, dtype=self.o_all.dtype).pin_memory()
+        s = self.stream
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(steps):
+                for k, h in host.items():
+                    self.dev[k].copy_(h, non_blocking=True)
+                self.graph.replay()
+                o_host.copy_(self.o_all, non_blocking=True)
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_s = max_over_ranks(e0.elapsed_time(e1)) / steps / 1e3
+        h2d = sum(h.numel() * h.element_size() for h in host.values())
+        return {"value": weak_scaling_throughput(self.bytes, world, e_s) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o_host.numel() * o_host.element_size()}
 
     def config(self):
         return workload_config(self.w.name)
@@ -656,7 +694,7 @@ def run_reference(args, rank, world):
         return
     from gated_deltanet_mixer_verify_b200.inputs import as_f64
     from oracle import gdn_oracle as orc
-    name = args.workload
+    name = "batched_verify" if args.workload == "all" else args.workload   # the headline's config
     if name == "prefill":
         sub = workload(name, T=256, H_k=1, H_v=3)
         f = as_f64(make_inputs(sub))
@@ -724,41 +762,10 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="batched_verify")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tokens", type=int, default=0,
-                    help="prefill only: prompt length override (default 32768), for profiling a "
-                         "smaller case")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        return
-
-    import datetime
-    import torch.distributed as dist
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    Prefill.tokens = args.tokens
-    wl = WORKLOADS[args.workload](args.workload, rank, dev)
+def measure(name, args, rank, world, dev, barrier, cpu_budget_s):
+    """Time K steps of one workload after W warm-ups (every rank), and return rank 0's record
+    (None on the other ranks)."""
+    wl = WORKLOADS[name](name, rank, dev)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -883,7 +890,7 @@ def main():
                 peak_source = "148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz"
             roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                         "frac": achieved / peak, "peak_source": peak_source,
-                        "traffic": ncu_traffic(args.workload), "kernel": wl.phase_kernel[k],
+                        "traffic": ncu_traffic(name), "kernel": wl.phase_kernel[k],
                         "algorithmic_flops_per_launch": wl.phase_work[k],
                         "phase_ms": dict(zip(wl.phase_names, phase_ms)),
                         "phase_timing": "each phase over the whole prompt, one after the other, in a "
@@ -912,7 +919,7 @@ def main():
             achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
             roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                         "frac": achieved / hbm_peak, "peak_source": "%s hbm_gbs (%s)" % (src, peak_kind),
-                        "traffic": ncu_traffic(args.workload),
+                        "traffic": ncu_traffic(name),
                         "algorithmic_bytes_per_launch": per_launch_bytes}
             dtype = "f32"
         line = {
@@ -930,14 +937,75 @@ def main():
             "e2e": e2e,
         }
         if not args.no_cpu_baseline and world == 1:
-            per_unit, units, desc, threads = oracle_sample(args.workload, 10.0)
-            cv, cu = cpu_value(args.workload, per_unit)
+            per_unit, units, desc, threads = oracle_sample(name, cpu_budget_s)
+            cv, cu = cpu_value(name, per_unit)
             line["cpu_baseline"] = {"value": cv, "unit": cu, "cores": threads, "kind": "oracle",
                                     "sample": desc}
-        print(json.dumps(line), flush=True)
 
     if isinstance(wl, (SingleSeq, ShortConv)):
         wl.graph = None
+    return line if rank == 0 else None
+
+
+# Workloads whose records the default run nests under "configs" beside the headline (batched
+# verify): the other model-scale configurations, then the next rows built on the same path.
+NESTED = ["decode", "prefill", "single_seq_verify", "commit_next_verify", "verify_gated",
+          "short_conv", "accept", "accept_greedy"]
+# keys of a nested record (the headline line carries the run-wide ones)
+NESTED_KEYS = ["value", "unit", "ms_per_step", "dtype", "config", "token_heads_per_s", "frac_of_spec_8TBps",
+               "roofline", "clocks", "gpu_launches", "e2e", "cpu_baseline"]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["all"] + sorted(WORKLOADS), default="all",
+                    help="all (default): batched_verify as the headline, the others nested "
+                         "under \"configs\"")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="prefill only: prompt length override (default 32768), for profiling a "
+                         "smaller case")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import datetime
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    Prefill.tokens = args.tokens
+    if args.workload != "all":
+        line = measure(args.workload, args, rank, world, dev, barrier, 10.0)
+    else:
+        line = measure("batched_verify", args, rank, world, dev, barrier, 10.0)
+        nested = {}
+        for name in NESTED:
+            torch.cuda.empty_cache()
+            rec = measure(name, args, rank, world, dev, barrier, 1.5)
+            if rank == 0:
+                nested[name] = {k: rec[k] for k in NESTED_KEYS if k in rec}
+        if rank == 0:
+            line["configs"] = nested
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         barrier()
         dist.destroy_process_group()

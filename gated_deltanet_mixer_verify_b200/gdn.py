@@ -132,6 +132,12 @@ def _ptr(t: Optional[torch.Tensor]):
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
+    # Kernels launch on the current device's stream with raw pointers: a tensor on another
+    # GPU would be read and written through a peer address by the wrong device.
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError("tensor is on %s but the current CUDA device is cuda:%d; call under "
+                         "torch.cuda.device(%s)" % (t.device, cur, t.device))
     return t.data_ptr()
 
 

@@ -41,3 +41,18 @@ def gpu_verify(gdn, xd: dict, accept_len, inplace=True, out_dtype=torch.float32,
                         out_dtype=out_dtype)
     torch.cuda.synchronize()
     return o, out
+
+
+def launched_kernels(fn):
+    """Run fn and return (its result, the names of the CUDA kernels it launched), from the
+    CUPTI kernel trace that torch.profiler collects."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        r = fn()
+        torch.cuda.synchronize()
+    return r, {e.name for e in prof.events()}
+
+
+def sm_count() -> int:
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count

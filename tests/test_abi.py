@@ -266,3 +266,31 @@ def test_binding_rejects_element_types_the_abi_does_not_take(gdn):
         gdn.decode_step(*args(), st.half())
     with pytest.raises(TypeError, match="state_out must be float32"):
         gdn.chunk_prefill(*args(), None, st.double())
+
+
+def test_binding_rejects_a_tensor_on_another_device(gdn, monkeypatch):
+    # Kernels run on the current device's stream: a tensor on another GPU is refused before
+    # its pointer is taken. Emulated on the CPU with a stand-in for a cuda:1 tensor while
+    # cuda:0 is current.
+    import torch
+
+    class OnDevice1:
+        is_cuda = True
+        device = torch.device("cuda", 1)
+
+        def is_contiguous(self):
+            return True
+
+        def data_ptr(self):
+            raise AssertionError("pointer taken before the device check")
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="cuda:1 but the current CUDA device is cuda:0"):
+        gdn._ptr(OnDevice1())
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+
+    class Ok(OnDevice1):
+        def data_ptr(self):
+            return 0x1000
+
+    assert gdn._ptr(Ok()) == 0x1000

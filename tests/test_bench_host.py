@@ -92,3 +92,27 @@ def test_accept_bytes_and_reference_arm(bench, name):
     assert out.returncode == 0, out.stderr[-2000:]
     d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
     assert d["config"]["workload"] == name and d["value"] > 0 and d["cpu_baseline"]["cores"] == 1
+
+
+def test_default_reference_arm_times_the_headline_config():
+    # the driver's reference call passes no --workload: the oracle runs on batched verify
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["config"]["workload"] == "batched_verify"
+
+
+def test_nested_records_cover_the_model_scale_configs(bench):
+    # the default run nests decode, prefill and the 48-layer single sequence beside the
+    # headline, each record with its own timing, roofline, clocks and end-to-end leg
+    assert bench.NESTED[:3] == ["decode", "prefill", "single_seq_verify"]
+    assert set(bench.NESTED) | {"batched_verify"} == set(bench.WORKLOADS)
+    for k in ("value", "unit", "ms_per_step", "roofline", "clocks", "e2e", "gpu_launches"):
+        assert k in bench.NESTED_KEYS
+    assert all(hasattr(bench.WORKLOADS[n], "e2e") or n in ("decode", "prefill", "accept", "accept_greedy",
+                                                           "commit_next_verify", "verify_gated")
+               for n in bench.NESTED)

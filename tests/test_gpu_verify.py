@@ -11,7 +11,20 @@ import pytest
 import torch
 
 from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload
-from gdn_helpers import TOL, TOL_BF16_OUT, gpu_verify, oracle_verify, rel_err, to_dev
+from gdn_helpers import (TOL, TOL_BF16_OUT, gpu_verify, launched_kernels, oracle_verify, rel_err, sm_count,
+                         to_dev)
+
+# The kernel the batched-verify benchmark times; it runs when d_k = d_v = 128, 2 <= T <= 8 and
+# there is at least one (sequence, value head) per SM.
+TC_KERNEL = "gdn_verify_tc_kernel"
+
+
+def on_tc_kernel(fn, B, H_v):
+    """Run fn (a verify call) and check that the tensor-core kernel is the one it launched."""
+    assert B * H_v >= sm_count(), (B, H_v, sm_count())
+    r, names = launched_kernels(fn)
+    assert any(TC_KERNEL in n for n in names), names
+    return r
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +87,8 @@ def test_decode_full_size(gdn):
 
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8, 9, 12, 16])
 def test_every_block_length_and_accept_count(gdn, T):
+    # 6 value heads per sequence: the CUDA-core kernels (T = 1 and 9..16 never reach the
+    # tensor-core kernel at any size).
     w = workload("batched_verify", B=T + 1, T=T, H_k=2, H_v=6, seed=77 + T)
     accept = np.arange(T + 1, dtype=np.int32)                # every L in 0..T once
     check(gdn, w, gates="gentle", accept=accept)
@@ -92,52 +107,90 @@ def test_fp32_inputs_bf16_outputs_and_scale(gdn):
     check(gdn, workload("batched_verify", B=4, seed=6), out_dtype=torch.bfloat16, tol=TOL_BF16_OUT)
 
 
+@pytest.mark.parametrize("T", [2, 3, 4, 5, 6, 7, 8])
+def test_tensor_core_kernel_every_block_length_and_accept_count(gdn, T):
+    # Model-scale heads (H_k = 16, H_v = 48) and at least one head per SM, so that the
+    # benchmarked tensor-core kernel runs; every L in 0..T, in place for even T.
+    B = max(T + 1, 4)
+    w = workload("batched_verify", B=B, T=T, seed=170 + T)
+    accept = np.array([t % (T + 1) for t in range(B)], np.int32)
+    x = make_inputs(w, gates="gentle", accept_len=accept)
+    o_ref, S_ref, _ = oracle_verify(x, accept)
+    xd = to_dev(x)
+    o, S = on_tc_kernel(lambda: gpu_verify(gdn, xd, accept, inplace=T % 2 == 0), B, w.H_v)
+    assert rel_err(o, o_ref) <= TOL and rel_err(S, S_ref) <= TOL
+    assert torch.equal(S[0], xd["S0"][0])                    # L = 0: the state as it was
+
+
 def test_rollback_is_bit_exact_in_and_out_of_place(gdn):
-    w = workload("batched_verify", B=3, seed=9)
-    x = make_inputs(w, accept_len=np.zeros(3, np.int32))
+    B = 4
+    w = workload("batched_verify", B=B, seed=9)
+    x = make_inputs(w, accept_len=np.zeros(B, np.int32))
     xd = to_dev(x)
     for inplace in (True, False):
-        _, S = gpu_verify(gdn, xd, np.zeros(3, np.int32), inplace=inplace)
+        _, S = on_tc_kernel(lambda: gpu_verify(gdn, xd, np.zeros(B, np.int32), inplace=inplace), B, w.H_v)
         assert torch.equal(S, xd["S0"])
 
 
 def test_out_of_range_accept_commits_nothing_and_flags(gdn):
+    B = 4
+    w = workload("batched_verify", B=B, seed=10)
+    x = make_inputs(w)
+    xd = to_dev(x)
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    L = np.array([-1, 9, 4, 8], np.int32)
+    o_ref, S_ref, bad = oracle_verify(x, L)
+    assert list(bad) == [1, 1, 0, 0]
+    for inplace in (True, False):
+        status.zero_()
+        o, S = on_tc_kernel(lambda: gpu_verify(gdn, xd, L, inplace=inplace, status=status), B, w.H_v)
+        assert int(status[0].item()) & 1 == 1
+        assert torch.equal(S[:2], xd["S0"][:2])
+        assert rel_err(S[2:], S_ref[2:]) <= TOL and rel_err(o, o_ref) <= TOL
+    status.zero_()
+    gpu_verify(gdn, xd, np.array([8, 0, 4, 1], np.int32), status=status)
+    assert int(status[0].item()) == 0
+
+
+def test_out_of_range_accept_on_the_small_kernels(gdn):
+    # 3 sequences x 48 heads is below one head per SM: the CUDA-core head kernel runs.
     w = workload("batched_verify", B=3, seed=10)
     x = make_inputs(w)
     xd = to_dev(x)
     status = torch.zeros(4, dtype=torch.int32, device="cuda")
     L = np.array([-1, 9, 4], np.int32)
     o_ref, S_ref, bad = oracle_verify(x, L)
-    assert list(bad) == [1, 1, 0]
     for inplace in (True, False):
         status.zero_()
         o, S = gpu_verify(gdn, xd, L, inplace=inplace, status=status)
         assert int(status[0].item()) & 1 == 1
         assert torch.equal(S[:2], xd["S0"][:2])
         assert rel_err(S[2], S_ref[2]) <= TOL and rel_err(o, o_ref) <= TOL
-    status.zero_()
-    gpu_verify(gdn, xd, np.array([8, 0, 4], np.int32), status=status)
-    assert int(status[0].item()) == 0
 
 
 def test_identity_gates_leave_state_bit_exact(gdn):
     # a = -1e4 gives alpha = 1 exactly and b = -1e4 gives beta = 0 exactly: S_L = S_0.
-    w = workload("batched_verify", B=2, seed=11, in_dtype="f32")
-    x = make_inputs(w, accept_len=np.array([8, 5], np.int32))
+    B = 4
+    L = np.array([8, 5, 1, 0], np.int32)
+    w = workload("batched_verify", B=B, seed=11, in_dtype="f32")
+    x = make_inputs(w, accept_len=L)
     x["a"].fill_(-1e4)
     x["b"].fill_(-1e4)
-    _, S = gpu_verify(gdn, to_dev(x), np.array([8, 5], np.int32), inplace=False)
+    xd = to_dev(x)
+    _, S = on_tc_kernel(lambda: gpu_verify(gdn, xd, L, inplace=False), B, w.H_v)
     assert torch.equal(S.cpu(), x["S0"])
 
 
 def test_write_then_read(gdn):
     # alpha = beta = 1 and q = k: o_t = S_t khat_t = v_t right after each write.
-    w = workload("batched_verify", B=2, seed=12, in_dtype="f32")
+    B = 4
+    w = workload("batched_verify", B=B, seed=12, in_dtype="f32")
     x = make_inputs(w)
     x["q"] = x["k"].clone()
     x["a"].fill_(-1e4)
     x["b"].fill_(1e4)
-    o, _ = gpu_verify(gdn, to_dev(x), x["accept_len"].numpy())
+    xd = to_dev(x)
+    o, _ = on_tc_kernel(lambda: gpu_verify(gdn, xd, x["accept_len"].numpy()), B, w.H_v)
     assert rel_err(o, x["v"].double().numpy()) <= 1e-5
 
 

@@ -129,6 +129,10 @@ bool head_kernel_applies(const VerifyArgs& a);
 // Tensor-core form (d_k = d_v = 128, T <= 8, at least one (sequence, head) per SM).
 bool tc_kernel_applies(const VerifyArgs& a, int num_sms);
 cudaError_t launch_verify_tc(const VerifyArgs& a, cudaStream_t stream);
+// Persistent warp-specialised tensor-core form: the same shapes, with the commit fused at
+// device accept counts (no stash, no previous-block commit, no gated norm).
+bool pipe_kernel_applies(const VerifyArgs& a, int num_sms);
+cudaError_t launch_verify_pipe(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_verify_head(const VerifyArgs& a, cudaStream_t stream);
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
 

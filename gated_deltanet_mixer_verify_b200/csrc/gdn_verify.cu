@@ -541,6 +541,7 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    if (pipe_kernel_applies(a, nsm)) return launch_verify_pipe(a, stream);
     if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);   // fuses the gated norm
     // Other kernels: the mixer writes o, then the gated norm runs over o in place.
     VerifyArgs m = a;

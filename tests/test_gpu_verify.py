@@ -14,16 +14,19 @@ from gated_deltanet_mixer_verify_b200.inputs import make_inputs, workload
 from gdn_helpers import (TOL, TOL_BF16_OUT, gpu_verify, launched_kernels, oracle_verify, rel_err, sm_count,
                          to_dev)
 
-# The kernel the batched-verify benchmark times; it runs when d_k = d_v = 128, 2 <= T <= 8 and
-# there is at least one (sequence, value head) per SM.
+# The tensor-core kernels run when d_k = d_v = 128, 2 <= T <= 8 and there is at least one
+# (sequence, value head) per SM: the persistent pipelined one (the kernel the batched-verify
+# benchmark times) for a fused commit at device accept counts, the one-CTA-per-head one for the
+# other forms (two-phase stash, commit-on-next-verify, gated norm).
+PIPE_KERNEL = "gdn_verify_pipe_kernel"
 TC_KERNEL = "gdn_verify_tc_kernel"
 
 
-def on_tc_kernel(fn, B, H_v):
-    """Run fn (a verify call) and check that the tensor-core kernel is the one it launched."""
+def on_tc_kernel(fn, B, H_v, kernel=PIPE_KERNEL):
+    """Run fn (a verify call) and check that `kernel` is the one it launched."""
     assert B * H_v >= sm_count(), (B, H_v, sm_count())
     r, names = launched_kernels(fn)
-    assert any(TC_KERNEL in n for n in names), names
+    assert any(kernel in n for n in names), names
     return r
 
 pytestmark = pytest.mark.gpu
@@ -204,8 +207,9 @@ def test_two_phase_commit_equals_fused(gdn):
     nbytes = gdn.stash_bytes(w.B, w.T, w.H_k, w.H_v, w.d_k, w.d_v)
     stash = torch.empty(nbytes // 4, dtype=torch.float32, device="cuda")
     state = xd["S0"].clone()
-    o = gdn.verify_step(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["A_log"], xd["dt_bias"],
-                        state, None, None, stash=stash)
+    o = on_tc_kernel(lambda: gdn.verify_step(xd["q"], xd["k"], xd["v"], xd["a"], xd["b"], xd["A_log"],
+                                             xd["dt_bias"], state, None, None, stash=stash),
+                     w.B, w.H_v, kernel=TC_KERNEL)
     torch.cuda.synchronize()
     assert torch.equal(state, xd["S0"])                      # phase 1 leaves the state alone
     Ld = torch.as_tensor(L).cuda()

@@ -44,7 +44,7 @@ NOMINAL_TF32_OVER_BF16 = 1.1 / 2.25     # dense tensor-core peaks, tf32 vs bf16
 _CSRC = "gated_deltanet_mixer_verify_b200/csrc/"
 _HEADERS = [_CSRC + f for f in ("gdn_tc.cuh", "gdn_device.cuh", "gdn_internal.cuh")]
 KERNEL_SOURCES = {
-    "batched_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
+    "batched_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_pipe.cu"] + _HEADERS,
     "commit_next_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "verify_gated": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
@@ -772,22 +772,20 @@ def measure(name, args, rank, world, dev, barrier, cpu_budget_s):
         wl.step()
     torch.cuda.synchronize(dev)
 
-    # timed region: K steps, device events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # timed region: K steps back to back between two device events on the launching stream
+    # (no event between steps: one would sit between consecutive launches and stretch them)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for i in range(args.steps):
-            ev[i][0].record(stream)
             wl.step()
-            ev[i][1].record(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    elapsed_ms = max_over_ranks(start.elapsed_time(end))
-    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    local_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(local_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # Per-kernel times where a step overlaps kernels on two streams (prefill: the scan of one
@@ -914,7 +912,7 @@ def measure(name, args, rank, world, dev, barrier, cpu_budget_s):
             value = weak_scaling_throughput(wl.bytes, world, ms_per_step / 1e3) / 1e9
             unit = "GB/s"
             calls = getattr(wl, "calls_per_step", wl.launches_per_step)   # acceptance: one call, two kernels
-            kernel_ms = statistics.mean(step_ms) / calls
+            kernel_ms = local_ms / args.steps / calls   # average launch duration over the timed region
             per_launch_bytes = wl.bytes / calls
             achieved = per_launch_bytes / (kernel_ms / 1e3) / 1e9
             roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",

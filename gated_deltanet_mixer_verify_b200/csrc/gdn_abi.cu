@@ -277,9 +277,8 @@ gdn_status gdn_commit_and_verify(const gdn_shape* shape, int32_t prev_T, const v
     x.stash = stash;
     x.always_commit = 0;
     cudaStream_t s0 = static_cast<cudaStream_t>(stream);
-    int dev = 0, nsm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int nsm = 0;
+    cudaError_t e = gdn::current_sm_count(&nsm);
     if (e != cudaSuccess) return launched(e, who);
     if (gdn::tc_kernel_applies(x, nsm) && prev_T <= 8) {
         // One pass over the state: the tensor-core kernel applies the previous stash on-chip.

@@ -6,7 +6,42 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gdn {
+
+// Streaming multiprocessors of the current device, asked of the runtime once per device.
+inline cudaError_t current_sm_count(int* nsm) {
+    static std::atomic<int> cache[64];   // 0: not asked yet
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *nsm = c;
+            return cudaSuccess;
+        }
+    }
+    e = cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev].store(*nsm, std::memory_order_relaxed);
+    return e;
+}
+
+// The dynamic shared memory a kernel may use, set once per (kernel, device): the attribute
+// belongs to the function on the current device.
+template <auto Kernel>
+inline cudaError_t ensure_smem_attr(int bytes) {
+    static std::atomic<uint64_t> done{0};   // bit d: set on device d
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 // Arguments of one verify / decode launch (layouts as in include/gdn.h).
 struct VerifyArgs {

@@ -695,9 +695,7 @@ inline unsigned char* ws_rec_of(const VerifyArgs& a, void* ws) {
 // Chunks [c0, c1) of every (sequence, key head).
 template <typename InT>
 cudaError_t launch_prep(const VerifyArgs& a, void* workspace, int c0, int c1, cudaStream_t stream) {
-    // Per call: the attribute belongs to the function on the current device.
-    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_prep_kernel<InT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(PrepSmem));
+    cudaError_t e = ensure_smem_attr<gdn_prefill_prep_kernel<InT>>((int)sizeof(PrepSmem));
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(c1 - c0), a.Hk, a.B);
     gdn_prefill_prep_kernel<InT><<<grid, kPrepThreads, sizeof(PrepSmem), stream>>>(a, ws_kq_of(a, workspace),
@@ -708,8 +706,7 @@ cudaError_t launch_prep(const VerifyArgs& a, void* workspace, int c0, int c1, cu
 // Chunks [c0, c1), from the state in a.state_in (zero when NULL) to a.state_out.
 template <typename InT, typename OutT>
 cudaError_t launch_scan(const VerifyArgs& a, void* workspace, int c0, int c1, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_scan_kernel<InT, OutT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem_bytes<InT>());
+    cudaError_t e = ensure_smem_attr<gdn_prefill_scan_kernel<InT, OutT>>((int)scan_smem_bytes<InT>());
     if (e != cudaSuccess) return e;
     CUtensorMap v_map;
     e = tc::encode_tmap_tokens(&v_map, a.v, sizeof(InT) == 2, DV, a.Hv, a.T, a.B, kC);

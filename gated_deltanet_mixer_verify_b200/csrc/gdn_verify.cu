@@ -537,9 +537,8 @@ cudaError_t launch_commit_dk(const CommitArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
-    int dev = 0, nsm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int nsm = 0;
+    cudaError_t e = current_sm_count(&nsm);
     if (e != cudaSuccess) return e;
     if (pipe_kernel_applies(a, nsm)) return launch_verify_pipe(a, stream);
     if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);   // fuses the gated norm

@@ -438,16 +438,10 @@ template <int TM, typename InT, typename OutT>
 cudaError_t launch_head_t(const VerifyArgs& a, cudaStream_t stream) {
     constexpr int RPT = TM >= 16 ? 1 : 2;
     constexpr size_t smem = sizeof(HeadSmem<TM, RPT>);
-    static bool configured = false;   // per process; the attribute is per function
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gdn_verify_head_kernel<TM, RPT, InT, OutT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    int dev = 0, nsm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = ensure_smem_attr<gdn_verify_head_kernel<TM, RPT, InT, OutT>>((int)smem);
+    if (e != cudaSuccess) return e;
+    int nsm = 0;
+    e = current_sm_count(&nsm);
     if (e != cudaSuccess) return e;
     // With fewer (sequence, head) items than resident CTAs, split each head's rows over 2 or
     // 4 CTAs (each redoes the small per-head algebra) so that more SMs pull state from HBM.

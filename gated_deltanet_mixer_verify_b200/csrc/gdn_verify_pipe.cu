@@ -680,15 +680,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <typename InT, typename OutT>
 cudaError_t launch_pipe_t(const VerifyArgs& a, cudaStream_t stream) {
     constexpr size_t smem = sizeof(PipeSmem);
-    cudaError_t e = cudaFuncSetAttribute(gdn_verify_pipe_kernel<InT, OutT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_attr<gdn_verify_pipe_kernel<InT, OutT>>((int)smem);
     if (e != cudaSuccess) return e;
     CUtensorMap smap;
     e = tc::encode_tmap_f32_sw128(&smap, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
     if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int nsm = 0;
+    e = current_sm_count(&nsm);
     if (e != cudaSuccess) return e;
     const int grid = std::min(a.B * a.Hv, nsm);
     gdn_verify_pipe_kernel<InT, OutT><<<grid, kThreads, smem, stream>>>(smap, a, 1);

@@ -658,16 +658,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 template <typename InT, typename OutT, bool PRE, bool NORM>
 cudaError_t launch_tc_t(const VerifyArgs& a, cudaStream_t stream) {
     constexpr size_t smem = sizeof(TcSmem);
-    // Per call: the attribute belongs to the function on the current device.
-    cudaError_t e = cudaFuncSetAttribute(gdn_verify_tc_kernel<InT, OutT, PRE, NORM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_attr<gdn_verify_tc_kernel<InT, OutT, PRE, NORM>>((int)smem);
     if (e != cudaSuccess) return e;
     CUtensorMap map;
     e = tc::encode_tmap_f32_sw128(&map, a.state_in, (uint64_t)a.B * a.Hv * DV, DK, DV);
     if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    int nsm = 0;
+    e = current_sm_count(&nsm);
     if (e != cudaSuccess) return e;
     VerifyArgs ap = a;
     ap.prefetch_ahead = 2 * nsm;   // two CTAs per SM are resident

@@ -125,20 +125,33 @@ def make_shape(B, T, H_k, H_v, d_k, d_v, in_dtype=torch.bfloat16, out_dtype=torc
                   float(l2_eps), float(scale), sw)
 
 
+def _ptrs(*ts):
+    """Device pointers of the given tensors (None stays None), after the checks the C ABI cannot
+    make on a bare pointer: a CUDA tensor, contiguous, on the current device (kernels launch on
+    the current device's stream, so a tensor on another GPU would be read and written through a
+    peer address by the wrong device). The current device is asked for once per call."""
+    cur = None
+    out = []
+    for t in ts:
+        if t is None:
+            out.append(None)
+            continue
+        if not t.is_cuda:
+            raise ValueError("expected a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError("expected a contiguous tensor")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        d = t.get_device()
+        if d != cur:
+            raise ValueError("tensor is on cuda:%d but the current CUDA device is cuda:%d; call under "
+                             "torch.cuda.device(%d)" % (d, cur, d))
+        out.append(t.data_ptr())
+    return out
+
+
 def _ptr(t: Optional[torch.Tensor]):
-    if t is None:
-        return None
-    if not t.is_cuda:
-        raise ValueError("expected a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError("expected a contiguous tensor")
-    # Kernels launch on the current device's stream with raw pointers: a tensor on another
-    # GPU would be read and written through a peer address by the wrong device.
-    cur = torch.cuda.current_device()
-    if t.device.index != cur:
-        raise ValueError("tensor is on %s but the current CUDA device is cuda:%d; call under "
-                         "torch.cuda.device(%s)" % (t.device, cur, t.device))
-    return t.data_ptr()
+    return _ptrs(t)[0]
 
 
 def _stream(stream) -> Optional[int]:
@@ -208,9 +221,8 @@ def verify_step(q, k, v, a, b, A_log, dt_bias, state_in, state_out=None, accept_
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     if accept_len is not None and state_out is None:
         state_out = state_in
-    _check(_load().gdn_verify_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
-                                   _ptr(A_log), _ptr(dt_bias), _ptr(state_in), _ptr(state_out),
-                                   _ptr(accept_len), _ptr(o), _ptr(stash), _stream(stream)))
+    _check(_load().gdn_verify_step(ctypes.byref(sh), *_ptrs(q, k, v, a, b, A_log, dt_bias, state_in, state_out,
+                                                           accept_len, o, stash), _stream(stream)))
     return o
 
 
@@ -223,8 +235,7 @@ def commit(state_in, stash, accept_len, T, H_k, d_k=None, state_out=None, status
     _types(f32=(("state_in", state_in), ("state_out", state_out), ("stash", stash)), i32=(("accept_len", accept_len),))
     if state_out is None:
         state_out = state_in
-    _check(_load().gdn_commit(ctypes.byref(sh), _ptr(state_in), _ptr(state_out), _ptr(stash),
-                              _ptr(accept_len), _stream(stream)))
+    _check(_load().gdn_commit(ctypes.byref(sh), *_ptrs(state_in, state_out, stash, accept_len), _stream(stream)))
     return state_out
 
 
@@ -240,9 +251,9 @@ def commit_and_verify(q, k, v, a, b, A_log, dt_bias, state, prev_stash, prev_acc
             i32=(("prev_accept_len", prev_accept_len), ("accept_len", accept_len)))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
-    _check(_load().gdn_commit_and_verify(ctypes.byref(sh), int(prev_T), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
-                                         _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state), _ptr(prev_stash),
-                                         _ptr(prev_accept_len), _ptr(accept_len), _ptr(o), _ptr(stash),
+    _check(_load().gdn_commit_and_verify(ctypes.byref(sh), int(prev_T),
+                                         *_ptrs(q, k, v, a, b, A_log, dt_bias, state, prev_stash,
+                                                prev_accept_len, accept_len, o, stash),
                                          _stream(stream)))
     return o
 
@@ -260,10 +271,8 @@ def verify_step_gated(q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept
         raise ValueError("norm_z must have v's shape and dtype")
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
-    _check(_load().gdn_verify_step_gated(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
-                                         _ptr(A_log), _ptr(dt_bias), _ptr(state_in), _ptr(state_out),
-                                         _ptr(accept_len), _ptr(norm_z), _ptr(norm_w), float(norm_eps), _ptr(o),
-                                         _ptr(stash), _stream(stream)))
+    ptrs = _ptrs(q, k, v, a, b, A_log, dt_bias, state_in, state_out, accept_len, norm_z, norm_w, o, stash)
+    _check(_load().gdn_verify_step_gated(ctypes.byref(sh), *ptrs[:12], float(norm_eps), *ptrs[12:], _stream(stream)))
     return o
 
 
@@ -306,8 +315,8 @@ def accept(target, tokens, draft=None, uniforms=None, temperature=1.0, workspace
         accept_len = torch.empty(B, dtype=torch.int32, device=target.device)
     if next_token is None:
         next_token = torch.empty(B, dtype=torch.int32, device=target.device)
-    _check(_load().gdn_accept(ctypes.byref(sh), _ptr(target), _ptr(draft), _ptr(tokens), _ptr(uniforms),
-                              _ptr(accept_len), _ptr(next_token), _ptr(workspace),
+    _check(_load().gdn_accept(ctypes.byref(sh),
+                              *_ptrs(target, draft, tokens, uniforms, accept_len, next_token, workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream)))
     return accept_len, next_token
 
@@ -339,9 +348,9 @@ def short_conv(q, k, v, conv_w, hist_in, hist_out=None, accept_len=None, outputs
     else:
         q_out = k_out = v_out = None
     _check(_load().gdn_short_conv(ctypes.byref(sh), int(conv_w.shape[1]) if conv_w is not None else
-                                  int(hist_in.shape[1]) + 1, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                                  _ptr(hist_in), _ptr(hist_out), _ptr(accept_len), _ptr(q_out), _ptr(k_out),
-                                  _ptr(v_out), _stream(stream)))
+                                  int(hist_in.shape[1]) + 1,
+                                  *_ptrs(q, k, v, conv_w, hist_in, hist_out, accept_len, q_out, k_out, v_out),
+                                  _stream(stream)))
     return (q_out, k_out, v_out) if outputs else None
 
 
@@ -352,8 +361,7 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale
     _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state", state),))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
-    _check(_load().gdn_decode_step(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
-                                   _ptr(A_log), _ptr(dt_bias), _ptr(state), _ptr(o),
+    _check(_load().gdn_decode_step(ctypes.byref(sh), *_ptrs(q, k, v, a, b, A_log, dt_bias, state, o),
                                    _stream(stream)))
     return o
 
@@ -377,9 +385,8 @@ def chunk_prefill(q, k, v, a, b, A_log, dt_bias, state_in=None, state_out=None, 
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(_load().gdn_chunk_prefill(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(v), _ptr(a),
-                                     _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(state_in),
-                                     _ptr(state_out), _ptr(o), _ptr(workspace), wbytes,
+    _check(_load().gdn_chunk_prefill(ctypes.byref(sh), chunk,
+                                     *_ptrs(q, k, v, a, b, A_log, dt_bias, state_in, state_out, o, workspace), wbytes,
                                      _stream(stream)))
     return o, state_out
 
@@ -399,8 +406,7 @@ def chunk_prefill_prepare(q, k, a, b, A_log, dt_bias, workspace, H_v=None, d_v=N
     d_v = d_k if d_v is None else d_v
     sh = make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
     _dtypes(q, a, b, A_log, dt_bias)
-    _check(_load().gdn_chunk_prefill_prepare(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(a), _ptr(b),
-                                             _ptr(A_log), _ptr(dt_bias), _ptr(workspace),
+    _check(_load().gdn_chunk_prefill_prepare(ctypes.byref(sh), chunk, *_ptrs(q, k, a, b, A_log, dt_bias, workspace),
                                              _nbytes(workspace), _stream(stream)))
 
 
@@ -419,8 +425,8 @@ def chunk_prefill_scan(v, workspace, H_k, state_in=None, state_out=None, o=None,
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     if state_out is None:
         state_out = torch.empty((B, H_v, d_v, d_k), dtype=torch.float32, device=v.device)
-    _check(_load().gdn_chunk_prefill_scan(ctypes.byref(sh), chunk, _ptr(v), _ptr(state_in), _ptr(state_out),
-                                          _ptr(o), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+    _check(_load().gdn_chunk_prefill_scan(ctypes.byref(sh), chunk, *_ptrs(v, state_in, state_out, o, workspace),
+                                          _nbytes(workspace), _stream(stream)))
     return o, state_out
 
 
@@ -443,8 +449,7 @@ def chunk_prefill_noalloc(q, k, v, a, b, A_log, dt_bias, state_in=None, state_ou
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     if state_out is None:
         state_out = torch.empty((B, H_v, d_v, d_k), dtype=torch.float32, device=v.device)
-    _check(_load().gdn_chunk_prefill_noalloc(ctypes.byref(sh), chunk, _ptr(q), _ptr(k), _ptr(v),
-                                             _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
-                                             _ptr(state_in), _ptr(state_out), _ptr(o),
+    _check(_load().gdn_chunk_prefill_noalloc(ctypes.byref(sh), chunk,
+                                             *_ptrs(q, k, v, a, b, A_log, dt_bias, state_in, state_out, o),
                                              _stream(stream)))
     return o, state_out

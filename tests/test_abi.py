@@ -276,10 +276,12 @@ def test_binding_rejects_a_tensor_on_another_device(gdn, monkeypatch):
 
     class OnDevice1:
         is_cuda = True
-        device = torch.device("cuda", 1)
 
         def is_contiguous(self):
             return True
+
+        def get_device(self):
+            return 1
 
         def data_ptr(self):
             raise AssertionError("pointer taken before the device check")

@@ -48,7 +48,7 @@ KERNEL_SOURCES = {
     "commit_next_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "verify_gated": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_tc.cu"] + _HEADERS,
     "decode": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
-    "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_head.cu"] + _HEADERS,
+    "single_seq_verify": [_CSRC + "gdn_verify.cu", _CSRC + "gdn_verify_rec.cu"] + _HEADERS,
     "prefill": [_CSRC + "gdn_prefill.cu", _CSRC + "gdn_prefill.cuh"] + _HEADERS,
     "short_conv": [_CSRC + "gdn_conv.cu"] + _HEADERS,
     "accept": [_CSRC + "gdn_accept.cu"] + _HEADERS,
@@ -242,7 +242,7 @@ def workload_config(name):
         c["state"] = "fp32 [B,H_v,d_v,d_k], updated in place"
     elif name == "single_seq_verify":
         c["accept_len"] = "one min(Geometric(0.25), 8) per round, device int32"
-        c["launch"] = "48 launches captured in one CUDA graph"
+        c["launch"] = "48 launches captured in one CUDA graph, each a programmatic dependent of the one before"
     else:
         c["chunk"] = w.chunk
         c["state_in"] = "zero"
@@ -482,9 +482,11 @@ class SingleSeq:
         self.stream = torch.cuda.Stream(dev)
 
     def _eager(self):
+        # Programmatic dependent launch: each layer's kernel stages its own state while the
+        # previous layer's runs (a layer's state was last written by its own previous call).
         for x in self.layers:
             self.gdn.verify_step(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"],
-                                 x["dt_bias"], x["state"], x["state"], x["accept_len"], x["o"])
+                                 x["dt_bias"], x["state"], x["state"], x["accept_len"], x["o"], pdl=True)
 
     def step(self):
         if self.graph is None:
@@ -775,9 +777,10 @@ def measure(name, args, rank, world, dev, barrier, cpu_budget_s):
     # timed region: K steps back to back between two device events on the launching stream
     # (no event between steps: one would sit between consecutive launches and stretch them)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(torch.cuda.current_device())   # NVML set up before, not inside, the idle gap
     barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with clk:
         start.record(stream)
         for i in range(args.steps):
             wl.step()

@@ -53,6 +53,8 @@ gdn_status check_shape(const gdn_shape* s, int max_T, const char* who) {
     if (s->status_word && !aligned16(s->status_word) &&
         (reinterpret_cast<uintptr_t>(s->status_word) & 3u) != 0)
         return fail(GDN_ERR_INVALID_ARG, "%s: status_word misaligned", who);
+    if (s->launch_flags & ~GDN_LAUNCH_PDL)
+        return fail(GDN_ERR_INVALID_ARG, "%s: launch_flags 0x%x has unknown bits", who, s->launch_flags);
     return GDN_OK;
 }
 
@@ -96,6 +98,7 @@ gdn::VerifyArgs make_args(const gdn_shape* s, const void* q, const void* k, cons
     x.l2_eps = s->l2_eps;
     x.scale = s->scale;
     x.status_word = s->status_word;
+    x.pdl = (s->launch_flags & GDN_LAUNCH_PDL) != 0;
     return x;
 }
 

@@ -75,6 +75,8 @@ struct VerifyArgs {
     const void* norm_z;
     const float* norm_w;
     float norm_eps;
+    // Programmatic dependent launch (GDN_LAUNCH_PDL): honoured by the one-CTA-per-head kernel.
+    int pdl;
 };
 
 // Arguments of the second phase of a two-phase commit.
@@ -160,6 +162,12 @@ cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);
+
+// Latency form for fewer (sequence, value head) pairs than SMs: the per-token recurrence on
+// 16-row state slices in registers (d_k = 128, d_v a multiple of 16, T <= 16, fused commit or
+// decode, no stash).
+bool rec_kernel_applies(const VerifyArgs& a, int num_sms);
+cudaError_t launch_verify_rec(const VerifyArgs& a, cudaStream_t stream);
 
 // Tensor-core form (d_k = d_v = 128, T <= 8, at least one (sequence, head) per SM).
 bool tc_kernel_applies(const VerifyArgs& a, int num_sms);

@@ -545,7 +545,9 @@ cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
     // Other kernels: the mixer writes o, then the gated norm runs over o in place.
     VerifyArgs m = a;
     m.norm_z = nullptr;
-    if (head_kernel_applies(m)) {
+    if (rec_kernel_applies(m, nsm)) {
+        e = launch_verify_rec(m, stream);
+    } else if (head_kernel_applies(m)) {
         e = launch_verify_head(m, stream);
     } else {
         switch (m.dk) {

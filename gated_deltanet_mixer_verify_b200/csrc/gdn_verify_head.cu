@@ -89,6 +89,24 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_head_kernel(const Veri
         fence_barrier_init();
         if ((int)blockIdx.x < n_items) request_quarters(blockIdx.x, 0, nq);
     }
+    // Programmatic dependent launch (a no-op in plain stream order): the next kernel on the
+    // stream may start now; this one brings its first item's q, k, v rows into L2 (the L2 is
+    // coherent, so a later write by the kernel before it is still seen), and waits for that
+    // kernel to complete before it reads any other input or writes anything.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (p.pdl && (int)blockIdx.x < n_items && tid < 3 * T) {
+        const int it = blockIdx.x;
+        const int hh = (it / nsplit) % p.Hv, bb = it / nsplit / p.Hv, gg = hh / (p.Hv / p.Hk);
+        const int t = tid / 3, which = tid % 3;
+        const size_t el = p.in_bf16 ? 2 : 4;
+        const char* base = static_cast<const char*>(which == 0 ? p.q : which == 1 ? p.k : p.v);
+        const size_t off = which < 2 ? (((size_t)bb * T + t) * p.Hk + gg) * DK : (((size_t)bb * T + t) * p.Hv + hh) * dv;
+        const uint32_t bytes = (uint32_t)((which < 2 ? DK : dv) * el) & ~15u;
+        const char* src = base + off * el;
+        // A bulk prefetch needs a 16-byte aligned start (v rows of odd d_v may not have one).
+        if (bytes && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) bulk_prefetch_l2(src, bytes);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     bool ok = true;
     uint32_t parity = 0;   // phase of every stage's barrier for the current item
@@ -454,8 +472,17 @@ cudaError_t launch_head_t(const VerifyArgs& a, cudaStream_t stream) {
     // (the hardware scheduler overlaps one CTA's algebra with the other resident CTA's
     // streaming); the kernel still loops, so a smaller grid stays correct.
     const int grid = heads * x.row_split;
-    gdn_verify_head_kernel<TM, RPT, InT, OutT><<<grid, kThreads, smem, stream>>>(x);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gdn_verify_head_kernel<TM, RPT, InT, OutT>, x);
 }
 
 template <typename InT, typename OutT>

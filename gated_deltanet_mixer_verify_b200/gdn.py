@@ -21,6 +21,7 @@ _LIB_PATH = os.path.join(_PKG, "libgdn.so")
 
 GDN_F32, GDN_BF16 = 0, 1
 STATUS_BAD_ACCEPT = 1
+GDN_LAUNCH_PDL = 1   # gdn_shape.launch_flags: programmatic dependent launch (include/gdn.h)
 
 
 class GdnError(RuntimeError):
@@ -36,7 +37,7 @@ class _Shape(ctypes.Structure):
                 ("H_v", ctypes.c_int32), ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
                 ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
                 ("l2_eps", ctypes.c_float), ("scale", ctypes.c_float),
-                ("status_word", ctypes.c_void_p)]
+                ("status_word", ctypes.c_void_p), ("launch_flags", ctypes.c_uint32)]
 
 
 class _AcceptShape(ctypes.Structure):
@@ -119,10 +120,10 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 
 def make_shape(B, T, H_k, H_v, d_k, d_v, in_dtype=torch.bfloat16, out_dtype=torch.float32,
-               l2_eps=1e-6, scale=1.0, status_word: Optional[torch.Tensor] = None) -> _Shape:
+               l2_eps=1e-6, scale=1.0, status_word: Optional[torch.Tensor] = None, launch_flags=0) -> _Shape:
     sw = status_word.data_ptr() if status_word is not None else None
     return _Shape(B, T, H_k, H_v, d_k, d_v, _dtype_code(in_dtype), _dtype_code(out_dtype),
-                  float(l2_eps), float(scale), sw)
+                  float(l2_eps), float(scale), sw, int(launch_flags))
 
 
 def _ptrs(*ts):
@@ -160,14 +161,14 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
 
-def _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype) -> _Shape:
+def _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype, launch_flags=0) -> _Shape:
     B, T, H_k, d_k = k.shape
     H_v, d_v = v.shape[2], v.shape[3]
     if q.shape != k.shape or v.shape[:2] != (B, T):
         raise ValueError("q, k [B,T,H_k,d_k] and v [B,T,H_v,d_v] disagree")
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share a dtype")
-    return make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word)
+    return make_shape(B, T, H_k, H_v, d_k, d_v, q.dtype, out_dtype, l2_eps, scale, status_word, launch_flags)
 
 
 def _types(f32=(), i32=()):
@@ -210,11 +211,12 @@ def chunk_prefill_pieces(T, chunk=64) -> int:
 
 def verify_step(q, k, v, a, b, A_log, dt_bias, state_in, state_out=None, accept_len=None, o=None,
                 stash=None, l2_eps=1e-6, scale=1.0, status_word=None, out_dtype=torch.float32,
-                stream=None):
+                stream=None, pdl=False):
     """One verify block: o for all T tokens; with ``accept_len`` the committed state S_L goes
     to ``state_out`` (default: in place into ``state_in``); without it, ``stash`` (a float32
-    CUDA tensor of stash_bytes()/4 elements) receives what :func:`commit` needs. Returns o."""
-    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+    CUDA tensor of stash_bytes()/4 elements) receives what :func:`commit` needs. ``pdl``:
+    programmatic dependent launch (GDN_LAUNCH_PDL in include/gdn.h). Returns o."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype, GDN_LAUNCH_PDL if pdl else 0)
     _dtypes(q, a, b, A_log, dt_bias, o, out_dtype,
             f32=(("state_in", state_in), ("state_out", state_out), ("stash", stash)), i32=(("accept_len", accept_len),))
     if o is None:
@@ -355,9 +357,10 @@ def short_conv(q, k, v, conv_w, hist_in, hist_out=None, accept_len=None, outputs
 
 
 def decode_step(q, k, v, a, b, A_log, dt_bias, state, o=None, l2_eps=1e-6, scale=1.0,
-                status_word=None, out_dtype=torch.float32, stream=None):
-    """One plain decoding token (T = 1): returns o and updates ``state`` in place."""
-    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype)
+                status_word=None, out_dtype=torch.float32, stream=None, pdl=False):
+    """One plain decoding token (T = 1): returns o and updates ``state`` in place. ``pdl``:
+    programmatic dependent launch (GDN_LAUNCH_PDL in include/gdn.h)."""
+    sh = _shape_from(q, k, v, status_word, l2_eps, scale, out_dtype, GDN_LAUNCH_PDL if pdl else 0)
     _dtypes(q, a, b, A_log, dt_bias, o, out_dtype, f32=(("state", state),))
     if o is None:
         o = torch.empty(v.shape, dtype=out_dtype, device=v.device)

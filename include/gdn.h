@@ -67,9 +67,9 @@
 extern "C" {
 #endif
 
-/* 7: prefill in pieces (gdn_chunk_prefill_pieces); 6: gdn_accept; 5: gated norm;
- * 4: gdn_short_conv; 3: commit-and-verify */
-#define GDN_ABI_VERSION 7
+/* 8: gdn_shape.launch_flags (GDN_LAUNCH_PDL); 7: prefill in pieces (gdn_chunk_prefill_pieces);
+ * 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
+#define GDN_ABI_VERSION 8
 
 typedef enum {
     GDN_OK = 0,
@@ -99,7 +99,24 @@ typedef struct {
     float l2_eps;            /* inside the square root of the q/k normalisation, e.g. 1e-6 */
     float scale;             /* multiplies qhat, e.g. 1.0 or 1/sqrt(d_k) */
     int32_t* status_word;    /* device int32 or NULL; bits GDN_STATUS_* are OR-ed in */
+    uint32_t launch_flags;   /* 0, or GDN_LAUNCH_PDL (below) */
 } gdn_shape;
+
+/*
+ * GDN_LAUNCH_PDL -- programmatic dependent launch for gdn_verify_step and gdn_decode_step on
+ * the two small-batch kernels: the latency kernel (fewer (sequence, value head) pairs than
+ * SMs, d_k = 128, T <= 16, fused commit) and the one-CTA-per-head kernel (the other small
+ * batches, T = 1 and T > 8). The tensor-core kernels launch in plain stream order whatever
+ * the flag says. The kernel may begin while the kernel launched just before it on the stream
+ * is still running: it requests its state (state_in) and prefetches its q, k, v rows into L2
+ * at once, and waits for that kernel to complete before it reads anything else or writes
+ * anything. The caller guarantees that the kernel launched just before on the same stream
+ * does not write state_in (in a layer loop each layer's state was last written by that
+ * layer's previous call, long done; a loop of calls on one state must not set the flag).
+ * It also lets the kernel after it start once its own inputs are staged. Works inside a
+ * CUDA-graph capture.
+ */
+#define GDN_LAUNCH_PDL 1u
 
 /*
  * gdn_verify_step -- one mixer pass over a verify block of T tokens (7 drafts +

@@ -90,8 +90,8 @@ def test_decode_full_size(gdn):
 
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8, 9, 12, 16])
 def test_every_block_length_and_accept_count(gdn, T):
-    # 6 value heads per sequence: the CUDA-core kernels (T = 1 and 9..16 never reach the
-    # tensor-core kernel at any size).
+    # 6 value heads per sequence: the small-batch latency kernel (T = 1 and 9..16 never reach
+    # the tensor-core kernels at any size).
     w = workload("batched_verify", B=T + 1, T=T, H_k=2, H_v=6, seed=77 + T)
     accept = np.arange(T + 1, dtype=np.int32)                # every L in 0..T once
     check(gdn, w, gates="gentle", accept=accept)
@@ -156,7 +156,7 @@ def test_out_of_range_accept_commits_nothing_and_flags(gdn):
 
 
 def test_out_of_range_accept_on_the_small_kernels(gdn):
-    # 3 sequences x 48 heads is below one head per SM: the CUDA-core head kernel runs.
+    # 3 sequences x 48 heads is below one head per SM: the small-batch latency kernel runs.
     w = workload("batched_verify", B=3, seed=10)
     x = make_inputs(w)
     xd = to_dev(x)
@@ -231,3 +231,25 @@ def test_empty_batch(gdn):
     o = gdn.verify_step(z(x["q"]), z(x["k"]), z(x["v"]), z(x["a"]), z(x["b"]), x["A_log"],
                         x["dt_bias"], z(x["S0"]), None, z(x["accept_len"]))
     assert o.shape[0] == 0
+
+
+@pytest.mark.parametrize("T", [1, 8, 16])
+def test_latency_kernel_single_sequence(gdn, T):
+    # One sequence of 48 heads (fewer heads than SMs): the latency kernel, checked against the
+    # oracle for every accept count of the block in place, and a bad count and a rollback out
+    # of place (bit for bit).
+    w = workload("single_seq_verify", T=T, seed=200 + T)
+    for L in range(T + 1):
+        x = make_inputs(w, gates="gentle", accept_len=np.array([L], np.int32))
+        o_ref, S_ref, _ = oracle_verify(x, x["accept_len"].numpy())
+        xd = to_dev(x)
+        (o, S), names = launched_kernels(lambda: gpu_verify(gdn, xd, np.array([L], np.int32), inplace=L > 0))
+        assert any("gdn_verify_rec_kernel" in n for n in names), names
+        if L == 0:
+            assert torch.equal(S, xd["S0"])
+        assert rel_err(o, o_ref) <= TOL and rel_err(S, S_ref) <= TOL, (T, L)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = make_inputs(w)
+    xd = to_dev(x)
+    o, S = gpu_verify(gdn, xd, np.array([T + 1], np.int32), inplace=False, status=status)
+    assert int(status.item()) & 1 == 1 and torch.equal(S, xd["S0"])

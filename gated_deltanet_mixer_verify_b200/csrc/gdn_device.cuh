@@ -175,6 +175,11 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Brings the L2 line holding address src into L2 (any alignment; no data reaches the thread).
+__device__ __forceinline__ void prefetch_l2_line(const void* src) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t done;
     asm volatile(

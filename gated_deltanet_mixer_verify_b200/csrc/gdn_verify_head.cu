@@ -90,9 +90,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_head_kernel(const Veri
         if ((int)blockIdx.x < n_items) request_quarters(blockIdx.x, 0, nq);
     }
     // Programmatic dependent launch (a no-op in plain stream order): the next kernel on the
-    // stream may start now; this one brings its first item's q, k, v rows into L2 (the L2 is
-    // coherent, so a later write by the kernel before it is still seen), and waits for that
-    // kernel to complete before it reads any other input or writes anything.
+    // stream may start now; this one brings its first item's q, k, v rows and gate inputs into
+    // L2 (the L2 is coherent, so a later write by the kernel before it is still seen), and waits
+    // for that kernel to complete before it reads any other input or writes anything.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (p.pdl && (int)blockIdx.x < n_items && tid < 3 * T) {
         const int it = blockIdx.x;
@@ -105,6 +105,21 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_verify_head_kernel(const Veri
         const char* src = base + off * el;
         // A bulk prefetch needs a 16-byte aligned start (v rows of odd d_v may not have one).
         if (bytes && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) bulk_prefetch_l2(src, bytes);
+    }
+    if (p.pdl && (int)blockIdx.x < n_items && tid >= kThreads - 32) {   // and its gate inputs
+        const int it = blockIdx.x;
+        const int hh = (it / nsplit) % p.Hv, bb = it / nsplit / p.Hv;
+        const int ln = tid - (kThreads - 32);
+        const size_t el = p.in_bf16 ? 2 : 4;
+        for (int t = ln; t < T; t += 32) {
+            const size_t gi = (((size_t)bb * T + t) * p.Hv + hh) * el;
+            prefetch_l2_line(static_cast<const char*>(p.a) + gi);
+            prefetch_l2_line(static_cast<const char*>(p.b) + gi);
+        }
+        if (ln == 0) {
+            prefetch_l2_line(p.A_log + hh);
+            prefetch_l2_line(p.dt_bias + hh);
+        }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
 

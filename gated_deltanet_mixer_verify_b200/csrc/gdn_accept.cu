@@ -10,13 +10,24 @@
 // n leading survivors: accept_len = n + 1; the next token is argmax p_n (greedy), else a draw
 // with u_0 from the residual max(0, p_n - q_n) (n < T-1) or from p_{T-1} (all survived).
 //
-// Kernel 1 (one CTA per logit row, target rows then draft rows): streams the row once with
+// Kernel 1 (one CTA per logit row, a sequence's target rows then its draft rows, sequences in
+// order, so that sequences are finished one after another): streams the row once with
 // 16-byte loads, keeping the maximum and its first index (greedy) or the online maximum and
 // sum of 2^(x log2(e) / tau - max) (sampled). The last CTA to finish a sequence's rows (a
-// fence, then an atomic counter: nobody waits) finds n and writes accept_len (and the greedy
-// next token). Kernel 2 (sampled; 8 CTAs per sequence): tile sums (256 logits a tile) of the
-// residual over row n; the last CTA of the sequence draws the token by inverse CDF, first over
-// the tile sums, then inside one tile with a warp scan. Both are HBM-bound.
+// fence, then an atomic counter: nobody waits) finds n, writes accept_len (and the greedy
+// next token) and raises the sequence's flag. Kernel 2 (sampled; 8 CTAs per sequence): tile
+// sums (256 logits a tile) of the residual over row n; the last CTA of the sequence draws the
+// token by inverse CDF, first over the tile sums, then inside one tile with a warp scan.
+// Kernel 2 is a programmatic dependent of kernel 1: it is launched once every CTA of kernel 1
+// has started (each releases it at entry), and each of its CTAs waits for its sequence's flag
+// rather than for the whole of kernel 1, so that the draws of the sequences already finished
+// overlap the rows still streaming. Kernel 1 never waits and all of its CTAs have started,
+// so every flag is raised and every wait ends (it is bounded all the same, with a status
+// bit). Run after kernel 1 in plain stream order, the draw took 28% of the call's time for
+// 10% of its bytes. (Measured and slower: one persistent kernel doing both phases, over equal
+// contiguous shares of the logits, over shares fed by bulk copies through a shared-memory
+// ring, or over a list of quarter-row and draw items walked in grid strides or taken by an
+// atomic ticket; each paid a row piece's fixed latency once per item in series.)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,27 +43,49 @@ constexpr int kRowThreads = 512;
 constexpr int kTile = 256;         // logits per tile of the residual draw (8 per lane of a warp)
 constexpr int kSplit = 8;          // CTAs per sequence in the residual pass
 constexpr int kSplitThreads = 256;
+constexpr int kGreedyPadBytes = 80 * 1024;   // two row CTAs per SM in greedy calls (see launch_accept)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kMaxPolls = 1u << 20;   // bound of a draw CTA's wait for its sequence (~0.1-1 s)
 
 using RowStat = AcceptRowStat;
 
+// Eight consecutive logits kept raw while their loads are in flight (bf16 pairs, not fp32),
+// widened where they are used.
 template <typename T>
-__device__ __forceinline__ void ld8l(const T* p, float (&x)[8]);
+struct Raw8;
 template <>
-__device__ __forceinline__ void ld8l<float>(const float* p, float (&x)[8]) {
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(p)), b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+struct Raw8<float> {
+    float4 a, b;
+};
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 u;
+};
+__device__ __forceinline__ void ld8raw(const float* p, Raw8<float>& r) {
+    r.a = __ldcs(reinterpret_cast<const float4*>(p));
+    r.b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
 }
-template <>
-__device__ __forceinline__ void ld8l<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+__device__ __forceinline__ void ld8raw(const __nv_bfloat16* p, Raw8<__nv_bfloat16>& r) {
+    r.u = __ldcs(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ void widen8(const Raw8<float>& r, float (&x)[8]) {
+    x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+    x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+}
+__device__ __forceinline__ void widen8(const Raw8<__nv_bfloat16>& r, float (&x)[8]) {
+    const uint32_t w[4] = {r.u.x, r.u.y, r.u.z, r.u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         x[2 * e] = __uint_as_float(w[e] << 16);
         x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
     }
+}
+__device__ __forceinline__ void fill8(Raw8<float>& r) {
+    r.a = r.b = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+}
+__device__ __forceinline__ void fill8(Raw8<__nv_bfloat16>& r) {
+    const uint32_t ninf = 0xff80ff80u;   // two bf16 -inf
+    r.u = make_uint4(ninf, ninf, ninf, ninf);
 }
 
 template <typename T>
@@ -110,34 +143,47 @@ __device__ void decide(const AcceptArgs& a, int b, int lane) {
     }
 }
 
-// One CTA per logit row (target rows, then draft rows): the row streamed once, four 8-logit
-// groups per thread in flight (addresses clamped into the row, values past its end masked, so
-// that no branch sits between the loads). The last row of a sequence (fence, then an atomic
-// counter: nothing waits) has warp 0 decide.
+__device__ __forceinline__ uint32_t ld_acquire(const int* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// One CTA per logit row (a sequence's target rows, then its draft rows): the row streamed
+// once, four 8-logit groups per thread in flight (addresses clamped into the row, values past
+// its end masked, so that no branch sits between the loads). The last row of a sequence
+// (fence, then an atomic counter: nothing waits) has warp 0 decide and raise the flag.
 template <typename LT>
 __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const AcceptArgs a) {
-    const int64_t r = blockIdx.x;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the draw kernel may launch
+    const int rows_per_seq = a.sampled ? 2 * a.T - 1 : a.T;
+    const int b = (int)(blockIdx.x / rows_per_seq), k = (int)(blockIdx.x % rows_per_seq);
     const int64_t ntarget = (int64_t)a.B * a.T;
+    const int64_t r = k < a.T ? (int64_t)b * a.T + k : ntarget + (int64_t)b * (a.T - 1) + (k - a.T);
     const LT* row = r < ntarget ? static_cast<const LT*>(a.target) + r * a.V
                                 : static_cast<const LT*>(a.draft) + (r - ntarget) * a.V;
-    const int b = r < ntarget ? (int)(r / a.T) : (int)((r - ntarget) / (a.T - 1));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float c = kLog2e / a.tau;
     float m = -INFINITY, s = 0.f;
     int arg = 0x7fffffff;
     for (int base = 8 * tid; base < a.V; base += 4 * 8 * kRowThreads) {
-        float x[4][8];
+        Raw8<LT> xr[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) ld8l<LT>(row + min(base + g * 8 * kRowThreads, a.V - 8), x[g]);
+        for (int g = 0; g < 4; ++g) ld8raw(row + min(base + g * 8 * kRowThreads, a.V - 8), xr[g]);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const int i = base + g * 8 * kRowThreads;
             if (i >= a.V) continue;
+            float x[8];
+            widen8(xr[g], x);
             if (!a.sampled) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    if (x[g][e] > m) {   // indices rise within a thread: strict > keeps the first
-                        m = x[g][e];
+                    if (x[e] > m) {   // indices rise within a thread: strict > keeps the first
+                        m = x[e];
                         arg = i + e;
                     }
             } else {
@@ -145,13 +191,13 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
                 // maximum grows (rarely, after a thread's first groups)
                 float lm = m;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[g][e] * c);
+                for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[e] * c);
                 if (lm > m) {
                     s *= exp2_approx(m - lm);   // 0 when m is still -inf
                     m = lm;
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) s += exp2_approx(x[g][e] * c - m);
+                for (int e = 0; e < 8; ++e) s += exp2_approx(x[e] * c - m);
             }
         }
     }
@@ -182,31 +228,37 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
         st->s = s;
         st->arg = arg;
         __threadfence();   // the statistics are visible before this row is counted
-        const int rows_per_seq = a.sampled ? 2 * a.T - 1 : a.T;
         last = atomicAdd(&a.counters[b], 1) == rows_per_seq - 1;
     }
     __syncthreads();
     if (!last || warp != 0) return;
     __threadfence();
     decide<LT>(a, b, lane);
+    if (lane == 0) {
+        __threadfence();
+        st_release(&a.decided[b], 1);
+    }
 }
 
-// Logits j .. j+7 of the target row (and the draft row) as raw values.
+// Logits j .. j+7 of the target row (and the draft row) as raw values; -inf past the row.
 template <typename LT>
-__device__ __forceinline__ void load_pair(const LT* pr, const LT* qr, int j, int V, float (&x)[8], float (&y)[8]) {
+__device__ __forceinline__ void load_pair(const LT* pr, const LT* qr, int j, int V, Raw8<LT>& x, Raw8<LT>& y) {
+    fill8(x);
+    fill8(y);
     if (j < V) {
-        ld8l<LT>(pr + j, x);
-        if (qr) ld8l<LT>(qr + j, y);
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = y[e] = -INFINITY;
+        ld8raw(pr + j, x);
+        if (qr) ld8raw(qr + j, y);
     }
 }
 
 // Residual (or target) weights from raw logits and the row statistics (pi, qi: the reciprocals
 // of the row sums).
-__device__ __forceinline__ void weights_of(const float (&x)[8], const float (&y)[8], bool resid, float c, float pm,
+template <typename LT>
+__device__ __forceinline__ void weights_of(const Raw8<LT>& xr, const Raw8<LT>& yr, bool resid, float c, float pm,
                                            float pi, float qm, float qi, float (&w)[8]) {
+    float x[8], y[8];
+    widen8(xr, x);
+    widen8(yr, y);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         float v = exp2_approx(x[e] * c - pm) * pi;
@@ -223,6 +275,27 @@ template <typename LT>
 __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const AcceptArgs a) {
     const int b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int ok_s;
+    if (tid == 0) {   // the sequence's counts (see the note at the top)
+        uint32_t polls = 0;
+        int ok = 1;
+        while (ld_acquire(&a.decided[b]) == 0) {
+            if (++polls > kMaxPolls) {
+                ok = 0;
+                break;
+            }
+            __nanosleep(128);
+        }
+        ok_s = ok;
+    }
+    __syncthreads();
+    if (!ok_s) {
+        if (tid == 0) {
+            if (a.status_word) atomicOr(a.status_word, kStatusWaitTimeout);
+            a.next_token[b] = 0;
+        }
+        return;
+    }
     const int n = __ldcg(&a.nsurv[b]);
     const int64_t prow = (int64_t)b * a.T + n;
     const LT* pr = static_cast<const LT*>(a.target) + prow * a.V;
@@ -242,7 +315,7 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
     float* tsum = a.tiles + (int64_t)b * ntiles;
     constexpr int kStride = kSplit * (kSplitThreads / 32);   // tiles between a warp's iterations
     for (int t0 = blockIdx.y + kSplit * warp; t0 < ntiles; t0 += 4 * kStride) {
-        float x[4][8], y[4][8];
+        Raw8<LT> x[4], y[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) load_pair<LT>(pr, qr, (t0 + k * kStride) * kTile + 8 * lane, a.V, x[k], y[k]);
 #pragma unroll
@@ -323,7 +396,8 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
         return;
     }
     const int j = tile * kTile + 8 * lane;
-    float x[8], y[8], w[8];
+    Raw8<LT> x, y;
+    float w[8];
     load_pair<LT>(pr, qr, j, a.V, x, y);
     weights_of(x, y, resid, c, pm, pi, qm, qs, w);
     float mine2 = 0.f;
@@ -356,32 +430,51 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled) {
     const size_t rows = (size_t)B * T + (sampled ? (size_t)B * (T - 1) : 0);
     const size_t ntiles = ((size_t)V + kTile - 1) / kTile;
-    return rows * sizeof(RowStat) /* stats */ + (size_t)2 * B * 4 /* counters */ + (size_t)B * 4 /* n */ +
+    return rows * sizeof(RowStat) /* stats */ + (size_t)3 * B * 4 /* counters, flags */ + (size_t)B * 4 /* n */ +
            (sampled ? (size_t)B * ntiles * 4 : 0) + 64;
 }
 
 cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream) {
     // Workspace: row statistics, the counters (rows done per sequence, draw CTAs done per
-    // sequence), n per sequence, the tile sums.
+    // sequence) and the sequences' flags, n per sequence, the tile sums.
     const size_t rows = (size_t)a.B * a.T + (a.sampled ? (size_t)a.B * (a.T - 1) : 0);
     unsigned char* w = static_cast<unsigned char*>(workspace);
     a.stats = reinterpret_cast<RowStat*>(w);
     w += rows * sizeof(RowStat);
     a.counters = reinterpret_cast<int*>(w);
-    w += (size_t)2 * a.B * 4;
+    a.decided = a.counters + 2 * (size_t)a.B;
+    w += (size_t)3 * a.B * 4;
     a.nsurv = reinterpret_cast<int*>(w);
     w += (size_t)a.B * 4;
     a.tiles = reinterpret_cast<float*>(w);
-    cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)2 * a.B * 4, stream);
+    cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)3 * a.B * 4, stream);
     if (e != cudaSuccess) return e;
-    if (a.bf16) gdn_accept_rows_kernel<__nv_bfloat16><<<(unsigned)rows, kRowThreads, 0, stream>>>(a);
-    else gdn_accept_rows_kernel<float><<<(unsigned)rows, kRowThreads, 0, stream>>>(a);
+    // Greedy calls reserve shared memory they do not use, so that at most two row CTAs share an
+    // SM: at three (the kernel's registers allow it), the 512 rows of a 64 x 8 block make 1.15
+    // waves on 148 SMs and the second runs nearly empty (0.047 against 0.041 ms). Sampled calls
+    // keep three: more loads in flight per SM, and the draws fill the last wave.
+    const int pad = a.sampled ? 0 : kGreedyPadBytes;
+    if (!a.sampled) {
+        e = a.bf16 ? ensure_smem_attr<gdn_accept_rows_kernel<__nv_bfloat16>>(kGreedyPadBytes)
+                   : ensure_smem_attr<gdn_accept_rows_kernel<float>>(kGreedyPadBytes);
+        if (e != cudaSuccess) return e;
+    }
+    if (a.bf16) gdn_accept_rows_kernel<__nv_bfloat16><<<(unsigned)rows, kRowThreads, pad, stream>>>(a);
+    else gdn_accept_rows_kernel<float><<<(unsigned)rows, kRowThreads, pad, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || !a.sampled) return e;
-    const dim3 dgrid(a.B, kSplit);
-    if (a.bf16) gdn_accept_draw_kernel<__nv_bfloat16><<<dgrid, kSplitThreads, 0, stream>>>(a);
-    else gdn_accept_draw_kernel<float><<<dgrid, kSplitThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B, kSplit);
+    cfg.blockDim = dim3(kSplitThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return a.bf16 ? cudaLaunchKernelEx(&cfg, gdn_accept_draw_kernel<__nv_bfloat16>, a)
+                  : cudaLaunchKernelEx(&cfg, gdn_accept_draw_kernel<float>, a);
 }
 
 }  // namespace gdn

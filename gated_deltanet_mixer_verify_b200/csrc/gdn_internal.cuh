@@ -149,9 +149,12 @@ struct AcceptArgs {
     int32_t* accept_len;         // [B] out
     int32_t* next_token;         // [B] out
     int32_t* status_word;
-    AcceptRowStat* stats;        // set by the launcher from the workspace: row statistics,
-    int* nsurv;                  // surviving drafts per sequence,
-    int* counters;               // [2 B]: rows done per sequence, draw CTAs done per sequence,
+    // Set by the launcher from the workspace:
+    AcceptRowStat* stats;        // row statistics
+    int* nsurv;                  // surviving drafts per sequence
+    int* counters;               // [2 B]: rows done per sequence, draw CTAs done per sequence
+    int* decided;                // [B] 1 once the sequence's counts are written (zeroed with
+                                 //     the counters)
     float* tiles;                // residual tile sums per sequence
 };
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled);

@@ -209,10 +209,10 @@ def test_accept_validates_on_the_host(gdn):
     lib = gdn.lib()
     fake = 0x100000
     need = gdn.accept_workspace_bytes(64, 8, 151936, True)
-    # row statistics (16 bytes a row: 8 target + 7 draft rows per sequence), two counters and n
-    # per sequence, tile sums (594 tiles of 256 logits)
-    assert need == 64 * 15 * 16 + 2 * 64 * 4 + 64 * 4 + 64 * 594 * 4 + 64
-    assert gdn.accept_workspace_bytes(64, 8, 151936, False) == 64 * 8 * 16 + 2 * 64 * 4 + 64 * 4 + 64
+    # row statistics (16 bytes a row: 8 target + 7 draft rows per sequence), two counters, a
+    # flag and n per sequence, tile sums (594 tiles of 256 logits)
+    assert need == 64 * 15 * 16 + 3 * 64 * 4 + 64 * 4 + 64 * 594 * 4 + 64
+    assert gdn.accept_workspace_bytes(64, 8, 151936, False) == 64 * 8 * 16 + 3 * 64 * 4 + 64 * 4 + 64
     assert gdn.accept_workspace_bytes(1, 8, (1 << 18) + 8, True) == 0
     call = lambda V=1024, T=8, sampled=1, tau=1.0, ws=fake, nbytes=1 << 30, draft=fake, u=fake, dtype=1: lib.gdn_accept(
         ctypes.byref(gdn._accept_shape(4, T, V, gdn.torch.bfloat16 if dtype else gdn.torch.float32, sampled, tau)),

@@ -11,7 +11,7 @@ __all__ = ["verify_step", "verify_step_gated", "commit", "commit_and_verify", "d
            "short_conv", "conv_channels", "gated_rmsnorm", "accept", "accept_workspace_bytes",
            "chunk_prefill", "chunk_prefill_prepare", "chunk_prefill_scan", "chunk_prefill_noalloc",
            "chunk_prefill_pieces", "prefill_workspace_bytes", "stash_bytes", "selftest_bounded_wait",
-           "make_shape", "lib", "GdnError", "library_path"]
+           "make_shape", "lib", "last_verify_kernel", "GdnError", "library_path"]
 
 
 def __getattr__(name):

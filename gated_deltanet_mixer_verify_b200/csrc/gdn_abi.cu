@@ -644,4 +644,6 @@ gdn_status gdn_selftest_bounded_wait(int32_t* status_word, uint32_t polls, void*
 
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
 
+const char* gdn_last_verify_kernel(void) { return gdn::last_verify_kernel(); }
+
 }  // extern "C"

@@ -116,6 +116,8 @@ struct ConvArgs {
 
 // Host launchers; return cudaSuccess or the launch error. Shapes are validated by the caller.
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream);
+// Name of the kernel the calling thread's last launch_verify chose ("" before the first).
+const char* last_verify_kernel();
 cudaError_t launch_short_conv(const ConvArgs& a, int K, bool bf16, cudaStream_t stream);
 
 // Gated RMS normalisation of rows of d elements (gdn_norm.cu). y may be x (in place).

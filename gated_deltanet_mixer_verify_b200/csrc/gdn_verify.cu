@@ -536,20 +536,33 @@ cudaError_t launch_commit_dk(const CommitArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+thread_local const char* g_last_verify_kernel = "";
+
+const char* last_verify_kernel() { return g_last_verify_kernel; }
+
 cudaError_t launch_verify(const VerifyArgs& a, cudaStream_t stream) {
     int nsm = 0;
     cudaError_t e = current_sm_count(&nsm);
     if (e != cudaSuccess) return e;
-    if (pipe_kernel_applies(a, nsm)) return launch_verify_pipe(a, stream);
-    if (tc_kernel_applies(a, nsm)) return launch_verify_tc(a, stream);   // fuses the gated norm
+    if (pipe_kernel_applies(a, nsm)) {
+        g_last_verify_kernel = "gdn_verify_pipe_kernel";
+        return launch_verify_pipe(a, stream);
+    }
+    if (tc_kernel_applies(a, nsm)) {
+        g_last_verify_kernel = "gdn_verify_tc_kernel";
+        return launch_verify_tc(a, stream);   // fuses the gated norm
+    }
     // Other kernels: the mixer writes o, then the gated norm runs over o in place.
     VerifyArgs m = a;
     m.norm_z = nullptr;
     if (rec_kernel_applies(m, nsm)) {
+        g_last_verify_kernel = "gdn_verify_rec_kernel";
         e = launch_verify_rec(m, stream);
     } else if (head_kernel_applies(m)) {
+        g_last_verify_kernel = "gdn_verify_head_kernel";
         e = launch_verify_head(m, stream);
     } else {
+        g_last_verify_kernel = "gdn_verify_kernel";
         switch (m.dk) {
             case 16: e = launch_verify_dk<16>(m, stream); break;
             case 32: e = launch_verify_dk<32>(m, stream); break;

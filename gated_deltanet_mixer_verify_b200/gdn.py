@@ -97,6 +97,8 @@ def _load():
     lib.gdn_last_error.restype = ctypes.c_char_p
     lib.gdn_abi_version.argtypes = []
     lib.gdn_abi_version.restype = ctypes.c_int32
+    lib.gdn_last_verify_kernel.argtypes = []
+    lib.gdn_last_verify_kernel.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -104,6 +106,11 @@ def _load():
 def lib():
     """The loaded ctypes library (raises ImportError if it was never built)."""
     return _load()
+
+
+def last_verify_kernel() -> str:
+    """Name of the kernel this thread's last verify / decode call launched (gdn_last_verify_kernel)."""
+    return _load().gdn_last_verify_kernel().decode()
 
 
 def _check(rc: int):

@@ -67,9 +67,9 @@
 extern "C" {
 #endif
 
-/* 8: gdn_shape.launch_flags (GDN_LAUNCH_PDL); 7: prefill in pieces (gdn_chunk_prefill_pieces);
+/* 9: gdn_last_verify_kernel; 8: gdn_shape.launch_flags (GDN_LAUNCH_PDL); 7: prefill in pieces (gdn_chunk_prefill_pieces);
  * 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
-#define GDN_ABI_VERSION 8
+#define GDN_ABI_VERSION 9
 
 typedef enum {
     GDN_OK = 0,
@@ -423,6 +423,14 @@ const char* gdn_last_error(void);
 
 /* GDN_ABI_VERSION of the built library. */
 int32_t gdn_abi_version(void);
+
+/*
+ * Name of the mixer kernel that the calling host thread's most recent gdn_verify_step,
+ * gdn_verify_step_gated, gdn_decode_step or gdn_commit_and_verify chose to launch (for
+ * example "gdn_verify_pipe_kernel"; "" before the first such call). The name is that of the
+ * CUDA kernel function. The string is static; the caller does not free it.
+ */
+const char* gdn_last_verify_kernel(void);
 
 #ifdef __cplusplus
 }

@@ -43,15 +43,26 @@ def gpu_verify(gdn, xd: dict, accept_len, inplace=True, out_dtype=torch.float32,
     return o, out
 
 
+# Runtime and profiler records a CUDA trace may hold besides kernels.
+_NOT_KERNELS = ("cuda", "Activity Buffer Request")
+
+
 def launched_kernels(fn):
     """Run fn and return (its result, the names of the CUDA kernels it launched), from the
-    CUPTI kernel trace that torch.profiler collects."""
+    CUPTI kernel trace that torch.profiler collects. Once in a long run the trace held the
+    runtime calls but no kernel record at all; fn cannot simply run again (many calls update
+    a state in place), so then the name comes from the library's own record of the kernel its
+    last verify or decode call chose (gdn_last_verify_kernel)."""
     from torch.profiler import ProfilerActivity, profile
+    from gated_deltanet_mixer_verify_b200 import gdn
     torch.cuda.synchronize()
     with profile(activities=[ProfilerActivity.CUDA]) as prof:
         r = fn()
         torch.cuda.synchronize()
-    return r, {e.name for e in prof.events()}
+    names = {e.name for e in prof.events()}
+    if not any(not n.startswith(_NOT_KERNELS) for n in names):
+        names.add(gdn.last_verify_kernel())
+    return r, names
 
 
 def sm_count() -> int:

@@ -153,8 +153,9 @@ __device__ __forceinline__ void st_release(int* p, int v) {
 }
 
 // One CTA per logit row (a sequence's target rows, then its draft rows): the row streamed
-// once, four 8-logit groups per thread in flight (addresses clamped into the row, values past
-// its end masked, so that no branch sits between the loads). The last row of a sequence
+// once, four 8-logit groups per thread in flight, the next four issued before the current
+// four are used (addresses clamped into the row, values past its end masked, so that no
+// branch sits between the loads). The last row of a sequence
 // (fence, then an atomic counter: nothing waits) has warp 0 decide and raise the flag.
 template <typename LT>
 __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const AcceptArgs a) {
@@ -169,10 +170,15 @@ __global__ void __launch_bounds__(kRowThreads) gdn_accept_rows_kernel(const Acce
     const float c = kLog2e / a.tau;
     float m = -INFINITY, s = 0.f;
     int arg = 0x7fffffff;
+    Raw8<LT> nx[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) ld8raw(row + min(8 * tid + g * 8 * kRowThreads, a.V - 8), nx[g]);
     for (int base = 8 * tid; base < a.V; base += 4 * 8 * kRowThreads) {
         Raw8<LT> xr[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) ld8raw(row + min(base + g * 8 * kRowThreads, a.V - 8), xr[g]);
+        for (int g = 0; g < 4; ++g) xr[g] = nx[g];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) ld8raw(row + min(base + 4 * 8 * kRowThreads + g * 8 * kRowThreads, a.V - 8), nx[g]);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const int i = base + g * 8 * kRowThreads;
@@ -450,9 +456,9 @@ cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)3 * a.B * 4, stream);
     if (e != cudaSuccess) return e;
     // Greedy calls reserve shared memory they do not use, so that at most two row CTAs share an
-    // SM: at three (the kernel's registers allow it), the 512 rows of a 64 x 8 block make 1.15
-    // waves on 148 SMs and the second runs nearly empty (0.047 against 0.041 ms). Sampled calls
-    // keep three: more loads in flight per SM, and the draws fill the last wave.
+    // SM whatever the register allocation: at three, the 512 rows of a 64 x 8 block make 1.15
+    // waves on 148 SMs and the second runs nearly empty (0.047 against 0.041 ms, measured when
+    // the kernel took 40 registers; it now takes 58, which also allows two).
     const int pad = a.sampled ? 0 : kGreedyPadBytes;
     if (!a.sampled) {
         e = a.bf16 ? ensure_smem_attr<gdn_accept_rows_kernel<__nv_bfloat16>>(kGreedyPadBytes)

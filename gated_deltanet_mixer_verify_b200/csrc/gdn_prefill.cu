@@ -848,12 +848,28 @@ cudaError_t launch_prefill(const VerifyArgs& a, int chunk, void* workspace, size
         cudaError_t e = launch_prefill_prepare(a, workspace, stream);
         return e == cudaSuccess ? launch_prefill_scan(a, workspace, stream) : e;
     }
+    auto bound = [&](int i) { return (int)((long long)nch * i / np); };
+    // Under stream capture the pieces run in order on the caller's stream, with the same
+    // bounds (so the same bits as an eager call). The side stream is shared by every caller on
+    // the device: joined to a capture, it would stay part of it until the capture ends, and an
+    // eager call from another thread in that window would queue into the capture.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return e;
+    if (cap != cudaStreamCaptureStatusNone) {
+        VerifyArgs ai = a;
+        for (int i = 0; i < np && e == cudaSuccess; ++i) {
+            if (i > 0) ai.state_in = a.state_out;
+            e = prepare_range(a, workspace, bound(i), bound(i + 1), stream);
+            if (e == cudaSuccess) e = scan_range(ai, workspace, bound(i), bound(i + 1), stream);
+        }
+        return e;
+    }
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
     PieceStreams* ps = nullptr;
-    cudaError_t e = piece_streams(&ps);
+    e = piece_streams(&ps);
     if (e != cudaSuccess) return e;
-    auto bound = [&](int i) { return (int)((long long)nch * i / np); };
     // Piece 0's preparation on the caller's stream, after the caller's earlier work.
     e = prepare_range(a, workspace, 0, bound(1), stream);
     if (e == cudaSuccess) e = cudaEventRecord(ps->ev[0], stream);

@@ -211,11 +211,12 @@ gdn_status gdn_commit_and_verify(const gdn_shape* shape, int32_t prev_T,
  * pieces of whole chunks. The scan of piece i runs on a stream of the greatest priority that
  * the library creates per device on first use (non-blocking), beside the preparation of piece
  * i + 1 on `stream`; events order the pieces and join that stream back to `stream` before the
- * call returns, so work queued on `stream` afterwards sees the finished o and state_out, and
- * the call can be captured into a CUDA graph like any other. The first such call on a device
- * creates the stream and its events, so make it outside stream capture. Calls from several
- * host threads are serialised while they queue their launches, and their scans share that
- * stream.
+ * call returns, so work queued on `stream` afterwards sees the finished o and state_out. The
+ * first such call on a device creates the stream and its events. Calls from several host
+ * threads are serialised while they queue their launches, and their scans share that stream.
+ * While `stream` is being captured into a CUDA graph, the pieces run in order on `stream`
+ * alone (same piece bounds, same results; the shared stream never joins a capture, so an
+ * eager call from another thread cannot land in the graph).
  */
 gdn_status gdn_chunk_prefill(const gdn_shape* shape, int32_t chunk,
                              const void* q, const void* k, const void* v,

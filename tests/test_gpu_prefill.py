@@ -154,8 +154,9 @@ def test_prefill_in_pieces_is_ordered_on_the_callers_stream(gdn):
 
 
 def test_prefill_in_pieces_captures_into_a_cuda_graph(gdn):
-    # The side stream joins the capture through the first event and leaves it through the
-    # last, so the 4-piece prefill replays as one graph with the eager call's bits.
+    # Under capture the 4 pieces run in order on the capture stream (the library's shared side
+    # stream never joins a capture), with the eager call's piece bounds: the replay gives the
+    # eager call's bits.
     w = workload("prefill", T=8192, H_k=2, H_v=6, seed=96, state_std=0.05)
     xd = to_dev(make_inputs(w, gates="gentle"))
     o_ref, s_ref = run_gpu(gdn, xd, xd["S0"])          # eager (also creates the side stream)

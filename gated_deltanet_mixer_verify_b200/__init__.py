@@ -10,7 +10,7 @@ any call into the mixer raises if the library is missing.
 __all__ = ["verify_step", "verify_step_gated", "commit", "commit_and_verify", "decode_step",
            "short_conv", "conv_channels", "gated_rmsnorm", "accept", "accept_workspace_bytes",
            "chunk_prefill", "chunk_prefill_prepare", "chunk_prefill_scan", "chunk_prefill_noalloc",
-           "chunk_prefill_pieces", "prefill_workspace_bytes", "stash_bytes", "selftest_bounded_wait",
+           "chunk_prefill_pieces", "prefill_workspace_bytes", "stash_bytes", "selftest_bounded_wait", "selftest_accept_wait",
            "make_shape", "lib", "last_verify_kernel", "GdnError", "library_path"]
 
 

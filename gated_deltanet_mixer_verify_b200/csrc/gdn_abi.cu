@@ -617,7 +617,7 @@ gdn_status gdn_accept(const gdn_accept_shape* shape, const void* target_logits, 
     if (!workspace || workspace_bytes < need)
         return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", who, need);
     if (!aligned16(workspace)) return fail(GDN_ERR_INVALID_ARG, "%s: workspace not 16-byte aligned", who);
-    gdn::AcceptArgs a;
+    gdn::AcceptArgs a = {};
     memset(&a, 0, sizeof(a));
     a.B = shape->B;
     a.T = shape->T;
@@ -640,6 +640,17 @@ gdn_status gdn_selftest_bounded_wait(int32_t* status_word, uint32_t polls, void*
         return fail(GDN_ERR_INVALID_ARG, "%s: status_word is NULL or misaligned", who);
     if (polls == 0 || polls > (1u << 20)) return fail(GDN_ERR_INVALID_ARG, "%s: polls must be 1..2^20", who);
     return launched(gdn::launch_bounded_wait_selftest(status_word, polls, static_cast<cudaStream_t>(stream)), who);
+}
+
+gdn_status gdn_selftest_accept_wait(int32_t* status_word, int32_t* next_token, uint32_t polls, void* stream) {
+    const char* who = "gdn_selftest_accept_wait";
+    if (!status_word || (reinterpret_cast<uintptr_t>(status_word) & 3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: status_word is NULL or misaligned", who);
+    if (!next_token || (reinterpret_cast<uintptr_t>(next_token) & 3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "%s: next_token is NULL or misaligned", who);
+    if (polls == 0 || polls > (1u << 20)) return fail(GDN_ERR_INVALID_ARG, "%s: polls must be 1..2^20", who);
+    return launched(gdn::launch_accept_wait_selftest(status_word, next_token, polls, static_cast<cudaStream_t>(stream)),
+                    who);
 }
 
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
         uint32_t polls = 0;
         int ok = 1;
         while (ld_acquire(&a.decided[b]) == 0) {
-            if (++polls > kMaxPolls) {
+            if (++polls > (a.max_polls ? a.max_polls : kMaxPolls)) {
                 ok = 0;
                 break;
             }
@@ -431,7 +431,30 @@ __global__ void __launch_bounds__(kSplitThreads) gdn_accept_draw_kernel(const Ac
     if (lane == 0) a.next_token[b] = (!fallback && first != 0x7fffffff) ? first : (lastp >= 0 ? lastp : 0);
 }
 
+// A flag that nothing raises, for the wait self-test.
+__device__ int g_never_raised = 0;
+
 }  // namespace
+
+cudaError_t launch_accept_wait_selftest(int32_t* status_word, int32_t* next_token, uint32_t polls,
+                                        cudaStream_t stream) {
+    // One sequence whose flag never rises: every draw CTA gives up after `polls` polls, sets
+    // the wait-timeout bit and writes next token 0, touching nothing else.
+    AcceptArgs a = {};
+    a.B = 1;
+    a.T = 2;
+    a.V = 8;
+    a.bf16 = true;
+    a.sampled = true;
+    a.tau = 1.f;
+    a.status_word = status_word;
+    a.next_token = next_token;
+    a.max_polls = polls;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.decided), g_never_raised);
+    if (e != cudaSuccess) return e;
+    gdn_accept_draw_kernel<__nv_bfloat16><<<dim3(1, kSplit), kSplitThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
 
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled) {
     const size_t rows = (size_t)B * T + (sampled ? (size_t)B * (T - 1) : 0);

@@ -157,6 +157,7 @@ struct AcceptArgs {
     int* counters;               // [2 B]: rows done per sequence, draw CTAs done per sequence
     int* decided;                // [B] 1 once the sequence's counts are written (zeroed with
                                  //     the counters)
+    uint32_t max_polls;          // bound of a draw CTA's wait for its flag (0: the default)
     float* tiles;                // residual tile sums per sequence
 };
 size_t accept_workspace_bytes(int B, int T, int V, bool sampled);
@@ -164,6 +165,9 @@ size_t accept_workspace_bytes(int B, int T, int V, bool sampled);
 // A bounded wait that nothing completes (gdn_selftest.cu).
 cudaError_t launch_bounded_wait_selftest(int32_t* status_word, uint32_t polls, cudaStream_t stream);
 cudaError_t launch_accept(AcceptArgs a, void* workspace, cudaStream_t stream);
+// The acceptance draw kernel alone, waiting `polls` polls on a flag that nothing raises.
+cudaError_t launch_accept_wait_selftest(int32_t* status_word, int32_t* next_token, uint32_t polls,
+                                        cudaStream_t stream);
 
 // One CTA per (sequence, value head) form for d_k = 128, d_v <= 128, T <= 16.
 bool head_kernel_applies(const VerifyArgs& a);

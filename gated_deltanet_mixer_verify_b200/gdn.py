@@ -73,6 +73,7 @@ def _load():
     lib.gdn_chunk_prefill_scan.argtypes = [S, ctypes.c_int32] + [_VP] * 5 + [ctypes.c_size_t, _VP]
     lib.gdn_short_conv.argtypes = [S, ctypes.c_int32] + [_VP] * 11
     lib.gdn_selftest_bounded_wait.argtypes = [_VP, ctypes.c_uint32, _VP]
+    lib.gdn_selftest_accept_wait.argtypes = [_VP, _VP, ctypes.c_uint32, _VP]
     A = ctypes.POINTER(_AcceptShape)
     lib.gdn_accept.argtypes = [A] + [_VP] * 7 + [ctypes.c_size_t, _VP]
     lib.gdn_accept_workspace_bytes.argtypes = [A]
@@ -83,7 +84,7 @@ def _load():
     for fn in ("gdn_verify_step", "gdn_commit", "gdn_decode_step", "gdn_commit_and_verify", "gdn_chunk_prefill",
                "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_prepare", "gdn_chunk_prefill_scan",
                "gdn_short_conv", "gdn_verify_step_gated", "gdn_gated_rmsnorm", "gdn_accept",
-               "gdn_selftest_bounded_wait"):
+               "gdn_selftest_bounded_wait", "gdn_selftest_accept_wait"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.gdn_stash_bytes.argtypes = [S]
     lib.gdn_stash_bytes.restype = ctypes.c_size_t
@@ -334,6 +335,13 @@ def selftest_bounded_wait(status_word, polls=1024, stream=None):
     """Run the library's bounded-wait failure path once: a wait that nothing completes gives up
     after `polls` polls and ORs the wait-timeout bit (2) into status_word (device int32)."""
     _check(_load().gdn_selftest_bounded_wait(_ptr(status_word), int(polls), _stream(stream)))
+
+
+def selftest_accept_wait(status_word, next_token, polls=1024, stream=None):
+    """Run the acceptance draw kernel's flag wait once with a flag nothing raises: it gives up
+    after `polls` polls, ORs the wait-timeout bit (2) into status_word and writes 0 to
+    next_token[0] (both device int32)."""
+    _check(_load().gdn_selftest_accept_wait(*_ptrs(status_word, next_token), int(polls), _stream(stream)))
 
 
 def conv_channels(H_k, H_v, d_k, d_v) -> int:

@@ -67,9 +67,9 @@
 extern "C" {
 #endif
 
-/* 9: gdn_last_verify_kernel; 8: gdn_shape.launch_flags (GDN_LAUNCH_PDL); 7: prefill in pieces (gdn_chunk_prefill_pieces);
+/* 10: gdn_selftest_accept_wait; 9: gdn_last_verify_kernel; 8: gdn_shape.launch_flags (GDN_LAUNCH_PDL); 7: prefill in pieces (gdn_chunk_prefill_pieces);
  * 6: gdn_accept; 5: gated norm; 4: gdn_short_conv; 3: commit-and-verify */
-#define GDN_ABI_VERSION 9
+#define GDN_ABI_VERSION 10
 
 typedef enum {
     GDN_OK = 0,
@@ -409,12 +409,23 @@ size_t gdn_chunk_prefill_workspace_bytes(const gdn_shape* shape, int32_t chunk);
 int32_t gdn_chunk_prefill_pieces(int64_t T, int32_t chunk);
 
 /*
- * gdn_selftest_bounded_wait -- test hook for the failure path that every bounded wait in the
- * library shares: one kernel waits, with the same helper, on an mbarrier that nothing completes;
+ * gdn_selftest_bounded_wait -- test hook for the failure path that every bounded mbarrier wait
+ * in the library shares: one kernel waits, with the same helper, on an mbarrier that nothing
+ * completes;
  * after `polls` polls (1..2^20) it gives up, ORs GDN_STATUS_WAIT_TIMEOUT into *status_word
  * (device int32) and returns. The context stays usable. Nothing faults, traps or hangs.
  */
 gdn_status gdn_selftest_bounded_wait(int32_t* status_word, uint32_t polls, void* stream);
+
+/*
+ * gdn_selftest_accept_wait -- test hook for the other kind of bounded wait: gdn_accept's draw
+ * kernel waits for its sequence's flag, raised by the row kernel's last row of the sequence.
+ * Here the draw kernel runs alone for one sequence whose flag nothing raises; each of its CTAs
+ * gives up after `polls` polls (1..2^20), ORs GDN_STATUS_WAIT_TIMEOUT into *status_word and
+ * writes 0 to next_token[0] (both device int32), and touches nothing else. The context stays
+ * usable. Nothing faults, traps or hangs.
+ */
+gdn_status gdn_selftest_accept_wait(int32_t* status_word, int32_t* next_token, uint32_t polls, void* stream);
 
 /* Static description of a status code. */
 const char* gdn_status_string(gdn_status status);

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     lib = gdn.lib()
-    assert lib.gdn_abi_version() == 9
+    assert lib.gdn_abi_version() == 10
     for code in (0, -1, -2, -3, -4):
         assert lib.gdn_status_string(code).decode().startswith("GDN_")
     assert "unknown" in lib.gdn_status_string(7).decode()

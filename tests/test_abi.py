@@ -296,3 +296,29 @@ def test_binding_rejects_a_tensor_on_another_device(gdn, monkeypatch):
             return 0x1000
 
     assert gdn._ptr(Ok()) == 0x1000
+
+
+def test_launch_flags_are_validated_on_the_host(gdn):
+    # GDN_LAUNCH_PDL (bit 0) is the only flag; any other bit is rejected before a launch, and
+    # the binding passes the flag through the shape.
+    INVALID = -1
+    assert gdn.GDN_LAUNCH_PDL == 1
+    sh = gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128, launch_flags=2)
+    assert sh.launch_flags == 2
+    assert _call_verify(gdn, sh) == INVALID
+    assert "launch_flags" in gdn.lib().gdn_last_error().decode()
+    sh = gdn.make_shape(B=2, T=8, H_k=16, H_v=48, d_k=128, d_v=128, launch_flags=gdn.GDN_LAUNCH_PDL | 4)
+    assert _call_verify(gdn, sh) == INVALID
+
+
+def test_selftests_validate_on_the_host(gdn):
+    INVALID = -1
+    lib = gdn.lib()
+    fake = 0x10000
+    assert lib.gdn_selftest_accept_wait(None, fake, 16, None) == INVALID
+    assert lib.gdn_selftest_accept_wait(fake, None, 16, None) == INVALID
+    assert lib.gdn_selftest_accept_wait(fake + 2, fake, 16, None) == INVALID      # misaligned
+    assert lib.gdn_selftest_accept_wait(fake, fake, 0, None) == INVALID
+    assert lib.gdn_selftest_accept_wait(fake, fake, (1 << 20) + 1, None) == INVALID
+    assert "polls" in lib.gdn_last_error().decode()
+    assert lib.gdn_selftest_bounded_wait(fake, 0, None) == INVALID
